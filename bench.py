@@ -1,0 +1,540 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged-attention hot path (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tv|reference]
+                    [--workload llama|mix|long|prefill|tiny]
+
+A step is one pass of the hot path over one batch:
+  llama / mix / tiny : tv_kv_append of one token per sequence, then
+                       tv_paged_decode over the whole paged context;
+  long               : tv_kv_append, tv_paged_decode_split (512-token
+                       partitions), tv_split_merge;
+  prefill            : tv_kv_append of the 512-token chunks, then
+                       tv_paged_prefill on the tensor cores.
+The default is the Llama-3.2-1B-shaped decode (64 sequences x 2048 tokens).
+Under torchrun every rank runs its own replica of the batch (sequences are
+independent; no collective touches the data path) and the whole-job value
+is the units of all ranks over the slowest rank's device time.
+
+--impl reference times the CPU oracle (double precision, the repository's
+correctness reference) on a bounded sample of the same workload; only rank 0
+runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("paged decode KV-read GB/s (% of B200 HBM peak) and "
+          "sequence-steps/s")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "measured")
+    except (OSError, KeyError, ValueError):
+        return (FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS,
+                "fallback")
+
+
+def _workload(name):
+    from paged_kv_cache_376_b200 import workloads as W
+    return {"llama": W.llama_decode, "mix": W.continuous_mix,
+            "long": W.long_split, "prefill": W.chunked_prefill,
+            "tiny": W.tiny_decode}[name]()
+
+
+def _config(wl, name):
+    cfg = {"workload": wl.name, "batch": wl.num_seqs,
+           "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
+           "head_dim": wl.head_dim, "page_size": wl.page_size,
+           "num_pages": wl.num_pages,
+           "context_tokens": int(wl.context_lens.sum())}
+    if name in ("llama", "mix", "tiny"):
+        cfg["step"] = "tv_kv_append + tv_paged_decode"
+    elif name == "long":
+        cfg["step"] = ("tv_kv_append + tv_paged_decode_split + "
+                       "tv_split_merge")
+        cfg["partition_tokens"] = wl.partition_tokens
+    else:
+        cfg["step"] = "tv_kv_append (512-token chunks) + tv_paged_prefill"
+        cfg["query_rows"] = int(wl.q.shape[0])
+    kvb = wl.kv_bytes_read()
+    cfg["l2"] = (f"inputs larger than L2: {kvb / 1e6:.0f} MB of K/V read per "
+                 "step, streamed with an L2 evict-first policy"
+                 if kvb > 126e6 else
+                 "working set smaller than L2 (latency configuration)")
+    return cfg
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+             "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu_index = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]),
+                             float(parts[3]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        busy = [r for r in rows if r[2] >= 50] or rows
+        reasons = sorted({self.NAMES[i] for r in busy
+                          for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(busy)}
+
+
+# ------------------------------------------------------------------ tv arm --
+
+class TVRunner:
+    """Device buffers and the calls of one step, marshalled once so that the
+    host submits a step in a few microseconds."""
+
+    def __init__(self, wl, name, device):
+        import torch
+        from paged_kv_cache_376_b200 import _lib
+        from paged_kv_cache_376_b200.device import upload
+        self.torch = torch
+        self.lib = _lib.load()
+        self.wl, self.name, self.device = wl, name, device
+        self.db = db = upload(wl, device)
+        self.out = torch.empty_like(db.q)
+        self.kind = ("prefill" if name == "prefill" else
+                     "split" if name == "long" else "decode")
+        if self.kind == "split":
+            maxp = wl.max_partitions()
+            b, hq, d = db.q.shape
+            self.po = torch.empty((b, hq, maxp, d), dtype=torch.float32,
+                                  device=device)
+            self.pl = torch.empty((b, hq, maxp), dtype=torch.float32,
+                                  device=device)
+            self.maxp = maxp
+        self.maxq = int(np.diff(wl.query_start_loc).max())
+        self.stream = torch.cuda.current_stream(device)
+
+    def _p(self, t):
+        import ctypes
+        return ctypes.c_void_p(t.data_ptr())
+
+    def step(self, timing=None):
+        """Launch one step on the current stream.  ``timing`` = (start, end)
+        events recorded around the dominant kernel."""
+        lib, db, wl = self.lib, self.db, self.wl
+        s = self.stream.cuda_stream
+        num_pages, ps, hkv, d = db.k_pool.shape
+        st = lib.tv_kv_append(
+            self._p(db.k_new), self._p(db.v_new), self._p(db.slot_mapping),
+            db.k_new.shape[0], self._p(db.k_pool), self._p(db.v_pool),
+            num_pages, hkv, d, ps, self._p(db.err), s)
+        assert st == 0, st
+        if timing is not None:
+            timing[0].record(self.stream)
+        b, hq = db.context_lens.shape[0], db.q.shape[1]
+        mb = db.block_tables.shape[1]
+        if self.kind == "decode":
+            st = lib.tv_paged_decode(
+                self._p(self.out), self._p(db.q), self._p(db.k_pool),
+                self._p(db.v_pool), self._p(db.block_tables), mb,
+                self._p(db.context_lens), b, hq, hkv, d, ps, num_pages,
+                wl.scale, self._p(db.err), s)
+        elif self.kind == "split":
+            st = lib.tv_paged_decode_split(
+                self._p(self.po), self._p(self.pl), self._p(db.q),
+                self._p(db.k_pool), self._p(db.v_pool),
+                self._p(db.block_tables), mb, self._p(db.context_lens), b, hq,
+                hkv, d, ps, num_pages, wl.scale, wl.partition_tokens,
+                self.maxp, self._p(db.err), s)
+        else:
+            st = lib.tv_paged_prefill(
+                self._p(self.out), self._p(db.q), db.q.shape[0],
+                self._p(db.query_start_loc), self._p(db.k_pool),
+                self._p(db.v_pool), self._p(db.block_tables), mb,
+                self._p(db.context_lens), b, self.maxq, hq, hkv, d, ps,
+                num_pages, wl.scale, self._p(db.err), s)
+        assert st == 0, st
+        if timing is not None:
+            timing[1].record(self.stream)
+        if self.kind == "split":
+            st = lib.tv_split_merge(
+                self._p(self.out), self._p(self.po), self._p(self.pl),
+                self._p(db.context_lens), b, hq, d, wl.partition_tokens,
+                self.maxp, s)
+            assert st == 0, st
+
+    def launches_per_step(self):
+        return 3 if self.kind == "split" else 2
+
+    # -- end to end: host inputs in, host result out, through the C ABI ------
+    def setup_e2e(self):
+        torch = self.torch
+        db = self.db
+        self.h_in = {}
+        for name in ("q", "k_new", "v_new", "slot_mapping", "block_tables",
+                     "context_lens", "query_start_loc"):
+            t = getattr(db, name)
+            self.h_in[name] = torch.empty(t.shape, dtype=t.dtype,
+                                          pin_memory=True).copy_(t.cpu())
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype,
+                                 pin_memory=True)
+
+    def e2e_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        d2h = self.h_out.numel() * self.h_out.element_size()
+        return h2d, d2h
+
+    def e2e_step(self):
+        db = self.db
+        for name, h in self.h_in.items():
+            getattr(db, name).copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+
+
+def _units(wl, name):
+    """(metric value numerator per step, unit, seq-steps per step)."""
+    if name == "prefill":
+        return wl.prefill_flops() / 1e12, "TFLOP/s", wl.num_seqs
+    return wl.kv_bytes_read() / 1e9, "GB/s", wl.num_seqs
+
+
+def run_tv(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    wl = _workload(args.workload)
+    runner = TVRunner(wl, args.workload, device)
+    per_step, unit, seqs = _units(wl, args.workload)
+    hbm, tfl, tfl_sus, peak_src = _peaks()
+    K, Wm = args.steps, args.warmup
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(device)
+
+    for _ in range(Wm):
+        runner.step()
+    barrier()
+
+    # ---- device-timed region ------------------------------------------------
+    ev = [(torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    gpu_index = _gpu_index(local_rank)
+    clocks = ClockSampler(gpu_index) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    wall0 = time.perf_counter()
+    t0.record()
+    for i in range(K):
+        runner.step(ev[i])
+    t1.record()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clock_info = clocks.stop() if clocks else None
+    ms = t0.elapsed_time(t1)
+    kern_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    ms_max = _max_over_ranks(ms, world, device)
+    kern_ms_max = _max_over_ranks(kern_ms, world, device)
+    err = int(runner.db.err.item())
+
+    # ---- end to end through the C ABI with host buffers -----------------------
+    runner.setup_e2e()
+    for _ in range(Wm):
+        runner.e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        runner.e2e_step()
+    e1.record()
+    barrier()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, device)
+    h2d, d2h = runner.e2e_bytes()
+
+    value = world * per_step * K / (ms_max / 1e3)
+    step_ms = ms_max / K
+    kern_per_launch = per_step / (kern_ms_max / 1e3)     # GB/s or TFLOP/s
+    if unit == "GB/s":
+        peak, bound, src = hbm, "hbm", peak_src
+    else:
+        peak, bound, src = tfl_sus, "tensor", peak_src
+    res = {
+        "metric": METRIC if args.workload != "prefill" else
+        "chunked prefill causal attention TFLOP/s (% of B200 bf16 peak)",
+        "value": round(value, 3), "unit": unit, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": round(step_ms, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, shuffled "
+        "page pool)",
+        "config": dict(_config(wl, args.workload),
+                       parallelism=f"replicas{world}" if world > 1
+                       else "single GPU"),
+        "seq_steps_per_s": round(world * seqs * K / (ms_max / 1e3), 1),
+        "hbm_frac" if unit == "GB/s" else "tensor_frac":
+            round(value / world / peak, 4),
+        "roofline": {
+            "bound": bound, "achieved": round(kern_per_launch, 2),
+            "peak": peak, "unit": unit, "frac": round(kern_per_launch / peak,
+                                                      4),
+            "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+            "kernel": {"decode": "tv_paged_decode", "split":
+                       "tv_paged_decode_split", "prefill":
+                       "tv_paged_prefill"}[runner.kind],
+            "kernel_ms": round(kern_ms_max, 6),
+            "traffic": None,
+        },
+        "e2e": {"value": round(world * per_step * K / (e2e_ms / 1e3), 3),
+                "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * runner.launches_per_step(),
+        "clocks": clock_info,
+        "device_error_word": err,
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, args.workload, budget_s=12.0)
+    return res
+
+
+def _gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+def _max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ oracle arm --
+
+def _oracle_step(wl, name, seqs):
+    """One oracle pass over the sequences ``seqs`` of the workload."""
+    import oracle
+    seqs = np.asarray(seqs)
+    if name == "prefill":
+        qsl = wl.query_start_loc
+        tok = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in seqs])
+        sl = wl.slot_mapping[tok]
+        kp, vp, _ = oracle.kv_append(wl.k_new[tok], wl.v_new[tok], sl,
+                                     wl.k_pool, wl.v_pool)
+        hq = wl.num_q_heads
+        ti = np.repeat(tok, hq).astype(np.int32)
+        hi = np.tile(np.arange(hq), len(tok)).astype(np.int32)
+        oracle.paged_prefill_rows(wl.q, qsl, kp, vp, wl.block_tables,
+                                  wl.context_lens, wl.scale, ti, hi)
+        return
+    kp, vp, _ = oracle.kv_append(wl.k_new[seqs], wl.v_new[seqs],
+                                 wl.slot_mapping[seqs], wl.k_pool, wl.v_pool)
+    hq = wl.num_q_heads
+    si = np.repeat(seqs, hq).astype(np.int32)
+    hi = np.tile(np.arange(hq), len(seqs)).astype(np.int32)
+    if name == "long":
+        o_p, lse = oracle.paged_decode_partials(
+            wl.q[seqs], kp, vp, wl.block_tables[seqs], wl.context_lens[seqs],
+            wl.scale, wl.partition_tokens, wl.max_partitions())
+        oracle.split_merge(o_p, lse, wl.context_lens[seqs],
+                           wl.partition_tokens)
+    else:
+        oracle.paged_decode_rows(wl.q, kp, vp, wl.block_tables,
+                                 wl.context_lens, wl.scale, si, hi)
+
+
+def _sample_work(wl, name, seqs):
+    if name == "prefill":
+        sub = 0
+        qsl, ctx = wl.query_start_loc, wl.context_lens
+        for s in seqs:
+            t = int(qsl[s + 1] - qsl[s])
+            p = int(ctx[s]) - t
+            sub += t * p + t * (t + 1) // 2
+        return 4 * wl.head_dim * wl.num_q_heads * sub / 1e12
+    per_tok = 2 * wl.num_kv_heads * wl.head_dim * 2
+    return float(wl.context_lens[np.asarray(seqs)].astype(np.int64).sum()
+                 * per_tok / 1e9)
+
+
+def _calibrate(wl, name, target_s):
+    """Smallest prefix of sequences whose oracle pass takes >= target_s
+    (or the whole batch)."""
+    n = 1
+    while True:
+        t = time.perf_counter()
+        _oracle_step(wl, name, range(n))
+        dt = time.perf_counter() - t
+        if dt >= target_s or n >= wl.num_seqs:
+            return n, dt
+        n = min(wl.num_seqs, max(n + 1, int(n * min(8.0, target_s /
+                                                     max(dt, 1e-3)))))
+
+
+def cpu_baseline(wl, name, budget_s=12.0):
+    import oracle
+    cores = oracle.max_threads()
+    n, _ = _calibrate(wl, name, budget_s / 4)
+    reps, total, t_all = 0, 0.0, time.perf_counter()
+    while reps < 1 or (time.perf_counter() - t_all < budget_s and reps < 5):
+        t = time.perf_counter()
+        _oracle_step(wl, name, range(n))
+        total += time.perf_counter() - t
+        reps += 1
+    work = _sample_work(wl, name, range(n))
+    unit = "TFLOP/s" if name == "prefill" else "GB/s"
+    return {"value": round(work * reps / total, 6), "unit": unit,
+            "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.num_seqs} sequences (all heads), "
+                      f"append + attention, {reps} pass(es), "
+                      f"{total:.1f} s of CPU time"}
+
+
+def run_reference(args):
+    import oracle
+    wl = _workload(args.workload)
+    cores = oracle.max_threads()
+    K, Wm = args.steps, args.warmup
+    # size the per-step sample so the whole run takes about two minutes
+    n, dt = _calibrate(wl, args.workload, 0.5)
+    per_seq = dt / n
+    n = int(max(1, min(wl.num_seqs, 120.0 / max(1, K + Wm) / per_seq)))
+    seqs = range(n)
+    for _ in range(Wm):
+        _oracle_step(wl, args.workload, seqs)
+    t = time.perf_counter()
+    for _ in range(K):
+        _oracle_step(wl, args.workload, seqs)
+    el = time.perf_counter() - t
+    work = _sample_work(wl, args.workload, seqs)
+    unit = "TFLOP/s" if args.workload == "prefill" else "GB/s"
+    value = work * K / el
+    sample = (f"{n} of {wl.num_seqs} sequences (all heads) per step, "
+              "append + attention")
+    return {
+        "metric": METRIC if args.workload != "prefill" else
+        "chunked prefill causal attention TFLOP/s (% of B200 bf16 peak)",
+        "value": round(value, 6), "unit": unit, "n_gpus": 1, "steps": K,
+        "warmup": Wm, "ms_per_step": round(el / K * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16, shuffled "
+        "page pool)", "config": _config(wl, args.workload),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": unit,
+                         "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit,
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["tv", "reference"], default="tv")
+    ap.add_argument("--workload", default="llama",
+                    choices=["llama", "mix", "long", "prefill", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    from paged_kv_cache_376_b200 import build as _build
+    _build.build()
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(
+            seconds=120), device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_tv(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * tv.h -- C ABI of libtv: PagedAttention over a block-table KV cache on B200.
+ *
+ * Operations, as the source pages define them:
+ *   [P1] "tiny-vllm：从零构建高性能LLM推理引擎的完整指南" (zingnex.cn), secs.
+ *        "PagedAttention：从操作系统借来的智慧" (fixed-size KV blocks located
+ *        through a per-sequence block table), "推理流程：从Prefill到Decode"
+ *        (decode appends the new token's K,V to the cache and attends over
+ *        it; prefill handles the prompt tokens in parallel), "在线Softmax：
+ *        数值稳定的注意力计算" (running max and correction factor), "Llama 3.2
+ *        1B架构拆解" (grouped-query attention, causal mask, softmax, weighted
+ *        sum of V), "BF16浮点数" (bf16 storage).
+ *   [P3] "Tiny-vLLM 实战：用 C++/CUDA 手写高性能 LLM 推理引擎" (hotdry.top),
+ *        secs. "内存池管理" (a page holds page_size x head_dim x num_kv_heads
+ *        bf16 values; pools are preallocated, no cudaMalloc during
+ *        inference), "CUDA Kernel 优化" item 3 (bf16 storage, fp32
+ *        accumulation).
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer owned by the caller; the
+ *     library allocates nothing and keeps no pointer after the call returns.
+ *   - bf16 tensors are passed as void* and hold IEEE bfloat16 bit patterns.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronise the host.
+ *   - Layouts (row-major, innermost last):
+ *       k_pool, v_pool   [num_pages][page_size][num_kv_heads][head_dim] bf16
+ *                        (slot s = page s / page_size, offset s % page_size)
+ *       block_tables     [num_seqs][max_blocks_per_seq] int32: physical page
+ *                        of logical block b = token positions [16b, 16b+16)
+ *       context_lens     [num_seqs] int32: tokens in the cache, counting the
+ *                        ones just appended
+ *       q, out (decode)  [num_seqs][num_q_heads][head_dim] bf16
+ *       q, out (prefill) [total_query_rows][num_q_heads][head_dim] bf16
+ *   - Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   - Supported: head_dim == 64, page_size == 16, num_q_heads a multiple of
+ *     num_kv_heads with a ratio in {1, 2, 4, 8}; every pointer 16-byte
+ *     aligned.  Anything else returns TV_ERR_UNSUPPORTED or
+ *     TV_ERR_INVALID_ARG before any launch.
+ *   - `err` (nullable) is a device uint32 word; kernels OR bits into it when
+ *     they meet bad data and skip that data instead of faulting:
+ *       TV_DEVERR_BAD_SLOT     slot_mapping entry >= num_pages * page_size
+ *       TV_DEVERR_BAD_PAGE     block-table entry outside [0, num_pages); the
+ *                              page's keys are left out
+ *       TV_DEVERR_BAD_CONTEXT  context_len < 0 or > max_blocks * page_size;
+ *                              clamped into range
+ *       TV_DEVERR_TIMEOUT      a bounded internal wait (2 s) ran out; the
+ *                              affected outputs are zeros
+ *       TV_DEVERR_BAD_QUERY    query_start_loc inconsistent with the context
+ *   - Outputs must not alias inputs.
+ *   - Return: TV_OK, or an error status; TV_ERR_CUDA means the launch failed
+ *     (tv_last_cuda_error() gives the CUDA error code).
+ */
+#ifndef TV_H_
+#define TV_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TV_OK = 0,
+  TV_ERR_INVALID_ARG = 1,
+  TV_ERR_UNSUPPORTED = 2,
+  TV_ERR_CUDA = 3
+} tv_status;
+
+enum {
+  TV_DEVERR_BAD_SLOT = 1u << 0,
+  TV_DEVERR_BAD_PAGE = 1u << 1,
+  TV_DEVERR_BAD_CONTEXT = 1u << 2,
+  TV_DEVERR_TIMEOUT = 1u << 3,
+  TV_DEVERR_BAD_QUERY = 1u << 4
+};
+
+/* Human-readable name of a status. Never NULL. */
+const char* tv_status_string(tv_status status);
+
+/* The CUDA error code of the last TV_ERR_CUDA returned on this thread. */
+int tv_last_cuda_error(void);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int tv_version(void);
+
+/*
+ * tv_kv_append -- write token t's K row and V row into pool slot
+ * slot_mapping[t] ([P1] "推理流程": append the new token's K,V to the cache;
+ * [P3] "内存池管理": page layout).
+ *   k_new, v_new   [num_tokens][num_kv_heads][head_dim] bf16, read only
+ *   slot_mapping   [num_tokens] int32; slot = page * page_size + offset;
+ *                  a negative slot is padding and is skipped; a slot beyond
+ *                  the pool is skipped and flagged TV_DEVERR_BAD_SLOT
+ *   k_pool, v_pool updated in place; every other byte is left unchanged
+ * The copy is bit-exact.  Two tokens mapped to one slot race (either may
+ * win).  num_tokens == 0 is a no-op.
+ */
+tv_status tv_kv_append(const void* k_new, const void* v_new,
+                       const int32_t* slot_mapping, int64_t num_tokens,
+                       void* k_pool, void* v_pool, int64_t num_pages,
+                       int num_kv_heads, int head_dim, int page_size,
+                       uint32_t* err, void* stream);
+
+/*
+ * tv_paged_decode -- one query per sequence at position context_lens[s]-1
+ * attends to keys 0 .. context_lens[s]-1 of its sequence, found through the
+ * block table ([P1] "PagedAttention", "推理流程", "在线Softmax", "Llama 3.2
+ * 1B架构拆解"):
+ *   out[s][h] = sum_j softmax_j(scale * q[s][h] . K_j) V_j
+ * with fp32 accumulation and one bf16 rounding (nearest even) of the result.
+ *   out            [num_seqs][num_q_heads][head_dim] bf16, written
+ *   q              [num_seqs][num_q_heads][head_dim] bf16
+ *   k_pool, v_pool [num_pages][page_size][num_kv_heads][head_dim] bf16
+ *   block_tables   [num_seqs][max_blocks_per_seq] int32; only the first
+ *                  ceil(context_lens[s] / page_size) entries are read
+ *   context_lens   [num_seqs] int32; 0 gives an all-zero output row
+ * Slots past a sequence's context (in its last page) are never used, so
+ * they may hold anything, NaN included.
+ */
+tv_status tv_paged_decode(void* out, const void* q, const void* k_pool,
+                          const void* v_pool, const int32_t* block_tables,
+                          int max_blocks_per_seq, const int32_t* context_lens,
+                          int num_seqs, int num_q_heads, int num_kv_heads,
+                          int head_dim, int page_size, int64_t num_pages,
+                          float scale, uint32_t* err, void* stream);
+
+/*
+ * tv_paged_decode_split -- tv_paged_decode restricted to logical key
+ * partitions p = [p*partition_tokens, (p+1)*partition_tokens) of each
+ * context (the blockwise online softmax of [P1] "在线Softmax"):
+ *   partial_out  [num_seqs][num_q_heads][max_partitions][head_dim] fp32:
+ *                the normalised attention over partition p alone
+ *   partial_lse  [num_seqs][num_q_heads][max_partitions] fp32: natural
+ *                log of sum_j exp(scale * q.K_j) over partition p
+ * An empty partition (p >= ceil(context / partition_tokens)) gets
+ * partial_out = 0 and partial_lse = -infinity.  partition_tokens must be a
+ * positive multiple of page_size; max_partitions >= the largest
+ * ceil(context_lens[s] / partition_tokens) the caller expects (partitions
+ * beyond max_partitions are not computed).
+ */
+tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
+                                const void* q, const void* k_pool,
+                                const void* v_pool,
+                                const int32_t* block_tables,
+                                int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs,
+                                int num_q_heads, int num_kv_heads,
+                                int head_dim, int page_size,
+                                int64_t num_pages, float scale,
+                                int partition_tokens, int max_partitions,
+                                uint32_t* err, void* stream);
+
+/*
+ * tv_split_merge -- combine the partials of tv_paged_decode_split:
+ *   M = max_p lse_p over p < min(ceil(context/partition_tokens),
+ *   max_partitions);  out = sum_p e^(lse_p - M) o_p / sum_p e^(lse_p - M)
+ *   out          [num_seqs][num_q_heads][head_dim] bf16, written
+ *   partial_out, partial_lse as written by tv_paged_decode_split
+ * A sequence with no keys gets a zero row.
+ */
+tv_status tv_split_merge(void* out, const float* partial_out,
+                         const float* partial_lse,
+                         const int32_t* context_lens, int num_seqs,
+                         int num_q_heads, int head_dim, int partition_tokens,
+                         int max_partitions, void* stream);
+
+/*
+ * tv_paged_prefill -- chunked prefill over the paged cache ([P1] "推理流程":
+ * prefill processes the prompt tokens in parallel under a causal mask).
+ * Sequence s owns query rows [query_start_loc[s], query_start_loc[s+1]);
+ * their K,V must already be in the cache (tv_kv_append).  With T_s rows and
+ * C = context_lens[s], row i sits at position C - T_s + i and attends to
+ * keys 0 .. C - T_s + i.  QK^T and PV run on the tcgen05 tensor cores (bf16
+ * in, fp32 accumulate in tensor memory); P is rounded to bf16 for PV.
+ *   out              [total_rows][num_q_heads][head_dim] bf16, written
+ *   q                [total_rows][num_q_heads][head_dim] bf16
+ *   num_query_rows   total_rows (the row count of q and out)
+ *   query_start_loc  [num_seqs + 1] int32, non-decreasing, [0] == 0,
+ *                    [num_seqs] <= num_query_rows
+ *   max_query_len    >= every T_s (sizes the grid); rows beyond a
+ *                    sequence's T_s are not touched
+ * A sequence with T_s > C is flagged TV_DEVERR_BAD_QUERY and skipped.
+ */
+tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
+                           const int32_t* query_start_loc, const void* k_pool,
+                           const void* v_pool, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* context_lens,
+                           int num_seqs, int max_query_len, int num_q_heads,
+                           int num_kv_heads, int head_dim, int page_size,
+                           int64_t num_pages, float scale, uint32_t* err,
+                           void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TV_H_ */

@@ -101,8 +101,10 @@ def kv_append(k_new, v_new, slot_mapping, k_pool, v_pool):
 
 
 def paged_decode_rows(q, k_pool, v_pool, block_tables, context_lens, scale,
-                      seq_idx, head_idx, with_lse=False):
-    """Decode attention for selected (sequence, q-head) rows; float64 [n][D]."""
+                      seq_idx, head_idx, with_lse=False, allow_bad=False):
+    """Decode attention for selected (sequence, q-head) rows; float64 [n][D].
+    Keys whose page id is outside the pool are left out; that raises unless
+    ``allow_bad``."""
     lib = _load()
     q = _c(q, np.uint16)
     kp, vp = _c(k_pool, np.uint16), _c(v_pool, np.uint16)
@@ -116,19 +118,20 @@ def paged_decode_rows(q, k_pool, v_pool, block_tables, context_lens, scale,
         _ptr(out), _ptr(lse), _ptr(si), _ptr(hi), si.shape[0], _ptr(q),
         _ptr(kp), _ptr(vp), _ptr(bt), bt.shape[1], _ptr(cl), hq, hkv, d,
         page_size, num_pages, float(scale))
-    if bad:
+    if bad and not allow_bad:
         raise ValueError(f"{bad} keys referenced pages outside the pool")
     return (out, lse) if with_lse else out
 
 
 def paged_decode(q, k_pool, v_pool, block_tables, context_lens, scale,
-                 with_lse=False):
+                 with_lse=False, allow_bad=False):
     """Decode attention for every (sequence, q-head): float64 [B][Hq][D]."""
     b, hq, d = q.shape
     seq_idx = np.repeat(np.arange(b, dtype=np.int32), hq)
     head_idx = np.tile(np.arange(hq, dtype=np.int32), b)
     res = paged_decode_rows(q, k_pool, v_pool, block_tables, context_lens,
-                            scale, seq_idx, head_idx, with_lse=True)
+                            scale, seq_idx, head_idx, with_lse=True,
+                            allow_bad=allow_bad)
     out = res[0].reshape(b, hq, d)
     return (out, res[1].reshape(b, hq)) if with_lse else out
 

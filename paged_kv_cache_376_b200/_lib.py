@@ -1,0 +1,218 @@
+"""ctypes binding of libtv (include/tv.h).
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of libtv.so.  Functions keep the C names and take torch tensors that
+already live on the GPU; they check dtype/shape/device, pass raw pointers and
+the current CUDA stream, and raise on a non-OK status.  There is no CPU or
+eager fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtv.so")
+
+TV_OK = 0
+STATUS = {0: "TV_OK", 1: "TV_ERR_INVALID_ARG", 2: "TV_ERR_UNSUPPORTED",
+          3: "TV_ERR_CUDA"}
+DEVERR_BAD_SLOT = 1 << 0
+DEVERR_BAD_PAGE = 1 << 1
+DEVERR_BAD_CONTEXT = 1 << 2
+DEVERR_TIMEOUT = 1 << 3
+DEVERR_BAD_QUERY = 1 << 4
+
+# (name, restype, argtypes) of every symbol include/tv.h declares
+_P, _I, _I64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+SIGNATURES = {
+    "tv_status_string": (ctypes.c_char_p, [_I]),
+    "tv_last_cuda_error": (_I, []),
+    "tv_version": (_I, []),
+    "tv_kv_append": (_I, [_P, _P, _P, _I64, _P, _P, _I64, _I, _I, _I, _P,
+                          _P]),
+    "tv_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                             _I64, _F, _P, _P]),
+    "tv_paged_decode_split": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I,
+                                   _I, _I, _I, _I64, _F, _I, _I, _P, _P]),
+    "tv_split_merge": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "tv_paged_prefill": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _I, _I,
+                              _I, _I, _I, _I, _I64, _F, _P, _P]),
+}
+
+_lib = None
+
+
+class TVError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libtv.so; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise TVError(
+            f"{path} is missing: build it with "
+            "`python -m paged_kv_cache_376_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != TV_OK:
+        lib = load()
+        extra = ""
+        if status == 3:
+            extra = f" (CUDA error {lib.tv_last_cuda_error()})"
+        raise TVError(f"{what}: {STATUS.get(status, status)}{extra}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def tv_kv_append(k_new, v_new, slot_mapping, k_pool, v_pool, err=None,
+                 stream=None):
+    """Scatter k_new/v_new [T][Hkv][D] (bf16) into pool slots
+    slot_mapping [T] (int32) of k_pool/v_pool [NP][PS][Hkv][D] in place."""
+    lib = load()
+    bf = torch.bfloat16
+    _cuda(k_new, bf, "k_new"), _cuda(v_new, bf, "v_new")
+    _cuda(k_pool, bf, "k_pool"), _cuda(v_pool, bf, "v_pool")
+    _cuda(slot_mapping, torch.int32, "slot_mapping")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    if v_pool.shape != k_pool.shape or k_new.shape != v_new.shape:
+        raise ValueError("K/V shape mismatch")
+    if k_new.shape[1:] != (hkv, d) or slot_mapping.shape != k_new.shape[:1]:
+        raise ValueError("k_new must be [T][Hkv][D] with slot_mapping [T]")
+    _check(lib.tv_kv_append(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+                            k_new.shape[0], _ptr(k_pool), _ptr(v_pool),
+                            num_pages, hkv, d, page_size, _ptr(err),
+                            _stream(stream)), "tv_kv_append")
+
+
+def tv_paged_decode(out, q, k_pool, v_pool, block_tables, context_lens,
+                    scale, err=None, stream=None):
+    """out[B][Hq][D] (bf16) = paged decode attention of q[B][Hq][D]."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_pool", k_pool),
+                 ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != b:
+        raise ValueError("shape mismatch")
+    _check(lib.tv_paged_decode(
+        _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), b, hq, hkv, d, page_size,
+        num_pages, float(scale), _ptr(err), _stream(stream)),
+        "tv_paged_decode")
+
+
+def tv_paged_decode_split(partial_out, partial_lse, q, k_pool, v_pool,
+                          block_tables, context_lens, scale,
+                          partition_tokens, err=None, stream=None):
+    """Per-partition fp32 partials: partial_out [B][Hq][P][D], partial_lse
+    [B][Hq][P] with P = partial_out.shape[2] partitions."""
+    lib = load()
+    bf = torch.bfloat16
+    _cuda(q, bf, "q"), _cuda(k_pool, bf, "k_pool"), _cuda(v_pool, bf, "v_pool")
+    _cuda(partial_out, torch.float32, "partial_out")
+    _cuda(partial_lse, torch.float32, "partial_lse")
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    maxp = partial_out.shape[2]
+    if partial_out.shape != (b, hq, maxp, d) or \
+            partial_lse.shape != (b, hq, maxp):
+        raise ValueError("partials must be [B][Hq][P][D] and [B][Hq][P]")
+    _check(lib.tv_paged_decode_split(
+        _ptr(partial_out), _ptr(partial_lse), _ptr(q), _ptr(k_pool),
+        _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), b, hq, hkv, d, page_size, num_pages, float(scale),
+        int(partition_tokens), maxp, _ptr(err), _stream(stream)),
+        "tv_paged_decode_split")
+
+
+def tv_split_merge(out, partial_out, partial_lse, context_lens,
+                   partition_tokens, stream=None):
+    """out[B][Hq][D] (bf16) = log-sum-exp merge of the partials."""
+    lib = load()
+    _cuda(out, torch.bfloat16, "out")
+    _cuda(partial_out, torch.float32, "partial_out")
+    _cuda(partial_lse, torch.float32, "partial_lse")
+    _cuda(context_lens, torch.int32, "context_lens")
+    b, hq, maxp, d = partial_out.shape
+    if out.shape != (b, hq, d):
+        raise ValueError("out must be [B][Hq][D]")
+    _check(lib.tv_split_merge(
+        _ptr(out), _ptr(partial_out), _ptr(partial_lse), _ptr(context_lens),
+        b, hq, d, int(partition_tokens), maxp, _stream(stream)),
+        "tv_split_merge")
+
+
+def tv_paged_prefill(out, q, query_start_loc, k_pool, v_pool, block_tables,
+                     context_lens, scale, max_query_len, err=None,
+                     stream=None):
+    """out[rows][Hq][D] (bf16) = chunked-prefill attention of q[rows][Hq][D]
+    over the paged cache (chunk K/V already appended)."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_pool", k_pool),
+                 ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    _cuda(query_start_loc, torch.int32, "query_start_loc")
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    rows, hq, _ = q.shape
+    b = context_lens.shape[0]
+    if out.shape != q.shape or query_start_loc.shape != (b + 1,):
+        raise ValueError("shape mismatch")
+    _check(lib.tv_paged_prefill(
+        _ptr(out), _ptr(q), rows, _ptr(query_start_loc), _ptr(k_pool),
+        _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), b, int(max_query_len), hq, hkv, d, page_size,
+        num_pages, float(scale), _ptr(err), _stream(stream)),
+        "tv_paged_prefill")

@@ -1,0 +1,70 @@
+// KV append: scatter each new token's K and V rows into their page slots.
+//
+// "tiny-vllm：从零构建高性能LLM推理引擎的完整指南", sec. "推理流程：从Prefill到
+// Decode": every generated token's K,V are computed and appended to the cache;
+// "Tiny-vLLM 实战：用 C++/CUDA 手写高性能 LLM 推理引擎", sec. "内存池管理": a
+// page holds page_size token rows of num_kv_heads x head_dim bf16 values.
+// Slot s names row s of the pool viewed as [num_pages * page_size][row]
+// (page s / page_size, offset s % page_size).  Negative slots are padding.
+//
+// The copy is bit-exact: one thread moves one 16-byte vector, so a token row
+// of 1 KB (8 heads x 64 x bf16) is 64 fully coalesced vectors per tensor.
+// The grid is a multiple of the SM count and strides over the work.
+#include "tv_device.cuh"
+#include "tv_kernels.h"
+
+namespace tv {
+namespace {
+
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(const uint4* __restrict__ k_new,
+                     const uint4* __restrict__ v_new,
+                     const int32_t* __restrict__ slot_mapping,
+                     int64_t num_tokens, uint4* __restrict__ k_pool,
+                     uint4* __restrict__ v_pool, int64_t num_slots,
+                     int row_vecs, uint32_t* err) {
+  const int64_t per_token = 2 * (int64_t)row_vecs;  // K vectors then V
+  const int64_t total = num_tokens * per_token;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int r = (int)(i - t * per_token);
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (r == 0) flag_error(err, DEVERR_BAD_SLOT);
+      continue;
+    }
+    if (r < row_vecs) {
+      k_pool[slot * row_vecs + r] = k_new[t * row_vecs + r];
+    } else {
+      const int c = r - row_vecs;
+      v_pool[slot * row_vecs + c] = v_new[t * row_vecs + c];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new,
+                             const int32_t* slot_mapping, int64_t num_tokens,
+                             void* k_pool, void* v_pool, int64_t num_slots,
+                             int row_bytes, uint32_t* err,
+                             cudaStream_t stream) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int row_vecs = row_bytes / 16;
+  const int64_t total = num_tokens * 2 * row_vecs;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (total + 255) / 256;
+  const int64_t cap = (int64_t)sms * 8;
+  const int blocks = (int)(want < cap ? want : cap);
+  kv_append_kernel<<<blocks, 256, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      slot_mapping, num_tokens, static_cast<uint4*>(k_pool),
+      static_cast<uint4*>(v_pool), num_slots, row_vecs, err);
+  return cudaGetLastError();
+}
+
+}  // namespace tv

@@ -1,0 +1,369 @@
+// Paged decode attention over a block-table KV cache, unsplit and split-KV.
+//
+// What it computes ("tiny-vllm：从零构建高性能LLM推理引擎的完整指南",
+// secs. "PagedAttention：从操作系统借来的智慧", "推理流程：从Prefill到Decode",
+// "在线Softmax：数值稳定的注意力计算", "Llama 3.2 1B架构拆解"): for every
+// sequence s and query head h, the single new query attends to the keys
+// 0 .. context_len-1 of its KV head h / G, found page by page through the
+// block table; softmax(scale * q.K) weights the V rows.  Storage is bf16,
+// every sum is fp32 ("Tiny-vLLM 实战：用 C++/CUDA 手写高性能 LLM 推理引擎",
+// sec. "CUDA Kernel 优化", item 3).
+//
+// B200 design.
+//  * One CTA per (KV head, sequence[, partition]).  Each K/V page slice it
+//    needs is 16 rows x 128 B (one KV head of a [page][16][Hkv][64] page) and
+//    is staged in shared memory by one 2-D TMA box per tensor, so the G query
+//    heads of the group reuse it from shared memory (GQA reuse).
+//  * Four warps per CTA, each with a private ring of kStages page slots and
+//    one mbarrier per slot; warp w takes pages w, w+4, w+8, ... so no warp
+//    ever waits for another until the final combine.  Block-table entries
+//    are prefetched 32 at a time, one per lane, ahead of the TMA issue.
+//  * Inside a warp: lane = 8*g + c; lane-group g owns tokens g, g+4, g+8,
+//    g+12 of the page, lane c owns head dims [8c, 8c+8).  QK partial dots
+//    are summed across the 8 lanes of a group with xor-shuffles; the softmax
+//    is online per page in base 2 (q is pre-scaled by scale*log2(e)): one
+//    max and one rescale per page, not per token.
+//  * The split variant writes the normalised partial output and the natural
+//    log-sum-exp of each 512-token (or any multiple of 16) partition; the
+//    merge kernel (split_merge.cu) combines them.
+#include "tv_device.cuh"
+#include "tv_kernels.h"
+
+namespace tv {
+namespace {
+
+constexpr int kD = 64;          // head_dim
+constexpr int kPS = 16;         // page_size
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowBytes = kD * 2;                 // one token, one KV head
+constexpr int kSliceBytes = kPS * kRowBytes;      // 2 KB
+constexpr int kStageBytes = 2 * kSliceBytes;      // K slice + V slice
+
+template <int kStages>
+struct DecodeSmem {
+  alignas(128) uint8_t ring[kWarps][kStages][kStageBytes];
+  alignas(8) uint64_t full[kWarps][kStages];
+};
+
+template <int G>
+struct Combine {  // per-warp results handed to the final combine
+  float m[kWarps][G];
+  float l[kWarps][G];
+  float acc[kWarps][G][kD];
+};
+
+template <int G, int kStages, bool kSplit>
+__global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
+    paged_decode_kernel(const DecodeArgs a,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v) {
+  static_assert(sizeof(Combine<G>) <= sizeof(DecodeSmem<kStages>::ring),
+                "combine buffer must fit in the ring");
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  // 1 KB of slack is requested at launch; align the carve-out by hand.
+  uint8_t* smem_raw = smem_dyn + ((1024 - (smem_u32(smem_dyn) & 1023)) & 1023);
+  auto& sm = *reinterpret_cast<DecodeSmem<kStages>*>(smem_raw);
+
+  const int kvh = blockIdx.x;
+  const int seq = blockIdx.y;
+  const int part = kSplit ? blockIdx.z : 0;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int grp = lane >> 3;   // token sub-group
+  const int chk = lane & 7;    // 16-byte chunk of the head dim
+
+  // ---- token range of this CTA --------------------------------------------
+  int ctx = a.context_lens[seq];
+  const int ctx_cap = a.max_blocks_per_seq * kPS;
+  if (ctx < 0 || ctx > ctx_cap) {
+    if (threadIdx.x == 0) flag_error(a.err, DEVERR_BAD_CONTEXT);
+    ctx = ctx < 0 ? 0 : ctx_cap;
+  }
+  int tok_begin = 0, tok_end = ctx;
+  if (kSplit) {
+    tok_begin = part * a.partition_tokens;
+    tok_end = min(ctx, tok_begin + a.partition_tokens);
+    if (tok_end < tok_begin) tok_end = tok_begin;
+  }
+  const int first_page = tok_begin / kPS;
+  const int n_pages = (tok_end - tok_begin + kPS - 1) / kPS;
+  // pages of this warp: first_page + warp + kWarps * i, i < my_n
+  const int my_n = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
+  const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq +
+                      first_page + warp;
+
+  // ---- barriers ------------------------------------------------------------
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&sm.full[warp][s]), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // ---- q for the G heads of this KV head, pre-scaled by scale*log2(e) -----
+  float qf[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint4 v = *reinterpret_cast<const uint4*>(
+        a.q + ((size_t)seq * a.num_q_heads + kvh * G + h) * kD + chk * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      qf[h][2 * i] = bf16_lo(w[i]) * a.scale_log2;
+      qf[h][2 * i + 1] = bf16_hi(w[i]) * a.scale_log2;
+    }
+  }
+
+  float m_run[G], l_run[G], acc[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_run[h] = -INFINITY;
+    l_run[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+  }
+
+  // Block-table entries of this warp's pages, 32 per batch, one per lane.
+  auto load_pids = [&](int batch) -> int {
+    const int i = batch * 32 + lane;
+    return i < my_n ? __ldg(bt + (size_t)i * kWarps) : 0;
+  };
+  int pid_cur = load_pids(0);
+  int pid_next = load_pids(1);
+  const uint64_t policy = l2_policy_evict_first();
+
+  auto issue = [&](int i, int pid, int stage) {
+    const bool ok = pid >= 0 && pid < a.num_pages;
+    if (!ok) flag_error(a.err, DEVERR_BAD_PAGE);
+    const int y = (ok ? pid : 0) * kPS;
+    const uint32_t bar = smem_u32(&sm.full[warp][stage]);
+    const uint32_t dst = smem_u32(&sm.ring[warp][stage][0]);
+    mbar_arrive_expect_tx(bar, kStageBytes);
+    tma_load_2d_hint(dst, &tm_k, kvh * kD, y, bar, policy);
+    tma_load_2d_hint(dst + kSliceBytes, &tm_v, kvh * kD, y, bar, policy);
+  };
+
+  // prologue: fill the ring
+#pragma unroll
+  for (int j = 0; j < kStages; ++j) {
+    const int pid = __shfl_sync(0xffffffffu, pid_cur, j);
+    if (lane == 0 && j < my_n) issue(j, pid, j);
+  }
+
+  bool failed = false;
+  int issued = min(my_n, kStages);
+  int i = 0;
+  for (; i < my_n; ++i) {
+    const int stage = i % kStages;
+    const uint32_t parity = (i / kStages) & 1;
+    if ((i & 31) == 0 && i > 0) {
+      pid_cur = pid_next;
+      pid_next = load_pids((i >> 5) + 1);
+    }
+    const int pid = __shfl_sync(0xffffffffu, pid_cur, i & 31);
+    const bool page_ok = pid >= 0 && pid < a.num_pages;
+    const int page_tok0 = (first_page + warp + kWarps * i) * kPS;
+
+    // Every lane observes the barrier (acquire of the TMA bytes); the
+    // outcome is made warp-uniform so the warp never diverges on it.
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(smem_u32(&sm.full[warp][stage]), parity))) {
+      failed = true;
+      break;
+    }
+    const uint8_t* kbase = &sm.ring[warp][stage][0];
+    const uint8_t* vbase = kbase + kSliceBytes;
+
+    // ---- scores for the 4 tokens of this lane group ------------------------
+    float s[4][G];
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int r = it * 4 + grp;
+      const uint4 kv =
+          *reinterpret_cast<const uint4*>(kbase + r * kRowBytes + chk * 16);
+      const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+      float kf[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        kf[2 * t] = bf16_lo(w[t]);
+        kf[2 * t + 1] = bf16_hi(w[t]);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d = fmaf(qf[h][e], kf[e], d);
+        s[it][h] = d;
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          s[it][h] += __shfl_xor_sync(0xffffffffu, s[it][h], off);
+      }
+      const bool valid = page_ok && (page_tok0 + r) < tok_end;
+#pragma unroll
+      for (int h = 0; h < G; ++h) s[it][h] = valid ? s[it][h] : -INFINITY;
+    }
+
+    // ---- online softmax, once per page -------------------------------------
+    float alpha[G], m_use[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float pm = fmaxf(fmaxf(s[0][h], s[1][h]), fmaxf(s[2][h], s[3][h]));
+      pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
+      pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
+      const float m_new = fmaxf(m_run[h], pm);
+      m_use[h] = m_new == -INFINITY ? 0.f : m_new;
+      alpha[h] = fast_exp2(m_run[h] - m_use[h]);
+      m_run[h] = m_new;
+      l_run[h] *= alpha[h];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[h][e] *= alpha[h];
+    }
+
+    // ---- P.V ----------------------------------------------------------------
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int r = it * 4 + grp;
+      const bool valid = page_ok && (page_tok0 + r) < tok_end;
+      uint4 vv =
+          *reinterpret_cast<const uint4*>(vbase + r * kRowBytes + chk * 16);
+      if (!valid) vv = make_uint4(0, 0, 0, 0);  // stale slots may hold NaN
+      const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+      float vf[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        vf[2 * t] = bf16_lo(w[t]);
+        vf[2 * t + 1] = bf16_hi(w[t]);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float p = fast_exp2(s[it][h] - m_use[h]);
+        l_run[h] += p;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(p, vf[e], acc[h][e]);
+      }
+    }
+
+    // ---- hand the slot back to the TMA unit ----------------------------------
+    fence_proxy_async_smem();
+    __syncwarp();
+    const int j = i + kStages;
+    const int src = ((j >> 5) == (i >> 5)) ? pid_cur : pid_next;
+    const int pid_j = __shfl_sync(0xffffffffu, src, j & 31);
+    if (j < my_n) {
+      if (lane == 0) issue(j, pid_j, stage);
+      ++issued;
+    }
+  }
+
+  if (failed) {
+    // Drain the copies this warp still has in flight (bounded), then wind
+    // down with an empty result.
+    if (lane == 0) flag_error(a.err, DEVERR_TIMEOUT);
+    for (int k = i; k < issued; ++k)
+      mbar_wait(smem_u32(&sm.full[warp][k % kStages]), (k / kStages) & 1);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      m_run[h] = -INFINITY;
+      l_run[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+    }
+  }
+
+  // ---- reduce over the 4 lane groups ----------------------------------------
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 8);
+      acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 16);
+    }
+  }
+  __syncthreads();  // every warp is done with its ring
+  auto& cb = *reinterpret_cast<Combine<G>*>(smem_raw);
+  if (grp == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cb.acc[warp][h][chk * 8 + e] = acc[h][e];
+      if (chk == 0) {
+        cb.m[warp][h] = m_run[h];
+        cb.l[warp][h] = l_run[h];
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- combine the 4 warps and write ------------------------------------------
+  for (int o = threadIdx.x; o < G * kD; o += kThreads) {
+    const int h = o / kD;
+    const int e = o % kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, cb.m[w][h]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = fast_exp2(cb.m[w][h] - M);
+        L = fmaf(cb.l[w][h], f, L);
+        O = fmaf(cb.acc[w][h][e], f, O);
+      }
+    }
+    const float out = L > 0.f ? O / L : 0.f;
+    const size_t head = (size_t)seq * a.num_q_heads + kvh * G + h;
+    if (kSplit) {
+      const size_t prow = head * a.max_partitions + part;
+      a.partial_out[prow * kD + e] = out;
+      if (e == 0)
+        a.partial_lse[prow] = L > 0.f ? (M + fast_log2(L)) * kLn2 : -INFINITY;
+    } else {
+      a.out[head * kD + e] = __float2bfloat16_rn(out);
+    }
+  }
+}
+
+template <int G, int kStages, bool kSplit>
+cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk,
+                     const CUtensorMap& tv, int num_kv_heads, int num_seqs,
+                     int parts, cudaStream_t stream) {
+  auto kern = paged_decode_kernel<G, kStages, kSplit>;
+  const int smem = sizeof(DecodeSmem<kStages>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(num_kv_heads, num_seqs, parts);
+  kern<<<grid, kThreads, smem, stream>>>(a, tk, tv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
+                                const CUtensorMap& tv, int num_kv_heads,
+                                int num_seqs, int group, bool split,
+                                int parts, cudaStream_t stream) {
+  constexpr int S = 3;
+  switch (group) {
+#define TV_CASE(G)                                                         \
+  case G:                                                                  \
+    return split ? launch_g<G, S, true>(a, tk, tv, num_kv_heads, num_seqs, \
+                                        parts, stream)                     \
+                 : launch_g<G, S, false>(a, tk, tv, num_kv_heads,          \
+                                         num_seqs, 1, stream);
+    TV_CASE(1)
+    TV_CASE(2)
+    TV_CASE(4)
+    TV_CASE(8)
+#undef TV_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tv

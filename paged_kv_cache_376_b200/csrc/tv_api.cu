@@ -1,0 +1,319 @@
+// C ABI of libtv (declared in include/tv.h): argument checks, TMA tensor-map
+// encoding and kernel launches.  Nothing here allocates device memory or
+// synchronises the host: the pool is the caller's preallocated memory
+// ("Tiny-vLLM 实战：用 C++/CUDA 手写高性能 LLM 推理引擎", sec. "内存池管理":
+// preallocate the pool, no cudaMalloc during inference).
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "tv.h"
+#include "tv_kernels.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kHeadDim = 64;
+constexpr int kPageSize = 16;
+
+tv_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return TV_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return TV_ERR_CUDA;
+}
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool group_ok(int num_q_heads, int num_kv_heads) {
+  if (num_q_heads <= 0 || num_kv_heads <= 0) return false;
+  if (num_q_heads % num_kv_heads) return false;
+  const int g = num_q_heads / num_kv_heads;
+  return g == 1 || g == 2 || g == 4 || g == 8;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library needs no link against libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The pool seen as a 2-D bf16 tensor [num_pages * page_size][Hkv * D]; the
+// box is one page of one KV head: 16 rows x 64 elements (128 B).
+tv_status pool_tensor_map(CUtensorMap* map, const void* pool,
+                          int64_t num_pages, int num_kv_heads,
+                          CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return TV_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)num_kv_heads * kHeadDim,
+                              (cuuint64_t)num_pages * kPageSize};
+  const cuuint64_t strides[1] = {(cuuint64_t)num_kv_heads * kHeadDim * 2};
+  const cuuint32_t box[2] = {kHeadDim, kPageSize};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return TV_ERR_CUDA;
+  }
+  return TV_OK;
+}
+
+// q seen as a 3-D bf16 tensor [rows][Hq][D]; the box is 32 rows x G heads x
+// 64 elements, i.e. the 4 query heads of one KV group for 32 query rows,
+// which land in shared memory as 128 rows of 128 B in (row, head) order.
+tv_status query_tensor_map(CUtensorMap* map, const void* q, int64_t rows,
+                           int num_q_heads, int group, int rows_per_box) {
+  auto fn = encode_fn();
+  if (!fn) return TV_ERR_CUDA;
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)num_q_heads,
+                              (cuuint64_t)(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2,
+                                 (cuuint64_t)num_q_heads * kHeadDim * 2};
+  const cuuint32_t box[3] = {kHeadDim, (cuuint32_t)group,
+                             (cuuint32_t)rows_per_box};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(q), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return TV_ERR_CUDA;
+  }
+  return TV_OK;
+}
+
+tv_status check_attention_shape(int num_q_heads, int num_kv_heads,
+                                int head_dim, int page_size) {
+  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (!group_ok(num_q_heads, num_kv_heads)) return TV_ERR_UNSUPPORTED;
+  return TV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tv_status_string(tv_status status) {
+  switch (status) {
+    case TV_OK: return "TV_OK";
+    case TV_ERR_INVALID_ARG: return "TV_ERR_INVALID_ARG";
+    case TV_ERR_UNSUPPORTED: return "TV_ERR_UNSUPPORTED";
+    case TV_ERR_CUDA: return "TV_ERR_CUDA";
+  }
+  return "TV_ERR_UNKNOWN";
+}
+
+int tv_last_cuda_error(void) { return g_last_cuda_error; }
+
+int tv_version(void) { return 100; }
+
+tv_status tv_kv_append(const void* k_new, const void* v_new,
+                       const int32_t* slot_mapping, int64_t num_tokens,
+                       void* k_pool, void* v_pool, int64_t num_pages,
+                       int num_kv_heads, int head_dim, int page_size,
+                       uint32_t* err, void* stream) {
+  if (num_tokens < 0 || num_pages <= 0 || num_kv_heads <= 0)
+    return TV_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return TV_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
+    return TV_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) ||
+      !aligned16(v_pool))
+    return TV_ERR_INVALID_ARG;
+  const int row_bytes = num_kv_heads * head_dim * 2;
+  return cuda_status(tv::launch_kv_append(
+      k_new, v_new, slot_mapping, num_tokens, k_pool, v_pool,
+      num_pages * page_size, row_bytes, err,
+      static_cast<cudaStream_t>(stream)));
+}
+
+static tv_status decode_common(void* out, float* partial_out,
+                               float* partial_lse, const void* q,
+                               const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables,
+                               int max_blocks_per_seq,
+                               const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim,
+                               int page_size, int64_t num_pages, float scale,
+                               int partition_tokens, int max_partitions,
+                               bool split, uint32_t* err, void* stream) {
+  tv_status st =
+      check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
+  if (st != TV_OK) return st;
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
+      !std::isfinite(scale))
+    return TV_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX)
+    return TV_ERR_UNSUPPORTED;
+  if (split && (partition_tokens <= 0 || partition_tokens % page_size ||
+                max_partitions <= 0 || max_partitions > 65535))
+    return TV_ERR_INVALID_ARG;
+  if (num_seqs == 0) return TV_OK;
+  if (!q || !k_pool || !v_pool || !block_tables || !context_lens)
+    return TV_ERR_INVALID_ARG;
+  if (split ? (!partial_out || !partial_lse || !aligned16(partial_out))
+            : !out)
+    return TV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+      (!split && !aligned16(out)))
+    return TV_ERR_INVALID_ARG;
+
+  CUtensorMap tk, tvm;
+  st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != TV_OK) return st;
+  st = pool_tensor_map(&tvm, v_pool, num_pages, num_kv_heads,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != TV_OK) return st;
+
+  tv::DecodeArgs a{};
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.partial_out = partial_out;
+  a.partial_lse = partial_lse;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.err = err;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_q_heads = num_q_heads;
+  a.num_pages = static_cast<int>(num_pages);
+  a.partition_tokens = split ? partition_tokens : 0;
+  a.max_partitions = split ? max_partitions : 1;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return cuda_status(tv::launch_paged_decode(
+      a, tk, tvm, num_kv_heads, num_seqs, num_q_heads / num_kv_heads, split,
+      split ? max_partitions : 1, static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_paged_decode(void* out, const void* q, const void* k_pool,
+                          const void* v_pool, const int32_t* block_tables,
+                          int max_blocks_per_seq, const int32_t* context_lens,
+                          int num_seqs, int num_q_heads, int num_kv_heads,
+                          int head_dim, int page_size, int64_t num_pages,
+                          float scale, uint32_t* err, void* stream) {
+  return decode_common(out, nullptr, nullptr, q, k_pool, v_pool, block_tables,
+                       max_blocks_per_seq, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, page_size,
+                       num_pages, scale, 0, 1, false, err, stream);
+}
+
+tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
+                                const void* q, const void* k_pool,
+                                const void* v_pool,
+                                const int32_t* block_tables,
+                                int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs,
+                                int num_q_heads, int num_kv_heads,
+                                int head_dim, int page_size,
+                                int64_t num_pages, float scale,
+                                int partition_tokens, int max_partitions,
+                                uint32_t* err, void* stream) {
+  return decode_common(nullptr, partial_out, partial_lse, q, k_pool, v_pool,
+                       block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, partition_tokens,
+                       max_partitions, true, err, stream);
+}
+
+tv_status tv_split_merge(void* out, const float* partial_out,
+                         const float* partial_lse,
+                         const int32_t* context_lens, int num_seqs,
+                         int num_q_heads, int head_dim, int partition_tokens,
+                         int max_partitions, void* stream) {
+  if (head_dim != kHeadDim) return TV_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || num_q_heads <= 0 || partition_tokens <= 0 ||
+      max_partitions <= 0)
+    return TV_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || num_q_heads > 65535) return TV_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return TV_OK;
+  if (!out || !partial_out || !partial_lse || !context_lens)
+    return TV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(partial_out)) return TV_ERR_INVALID_ARG;
+  return cuda_status(tv::launch_split_merge(
+      static_cast<__nv_bfloat16*>(out), partial_out, partial_lse,
+      context_lens, num_seqs, num_q_heads, partition_tokens, max_partitions,
+      static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
+                           const int32_t* query_start_loc, const void* k_pool,
+                           const void* v_pool, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* context_lens,
+                           int num_seqs, int max_query_len, int num_q_heads,
+                           int num_kv_heads, int head_dim, int page_size,
+                           int64_t num_pages, float scale, uint32_t* err,
+                           void* stream) {
+  tv_status st =
+      check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
+  if (st != TV_OK) return st;
+  if (num_q_heads / num_kv_heads != 4) return TV_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
+      max_query_len < 0 || num_query_rows < 0 || !std::isfinite(scale))
+    return TV_ERR_INVALID_ARG;
+  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX)
+    return TV_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || max_query_len == 0 || num_query_rows == 0)
+    return TV_OK;
+  if (!out || !q || !query_start_loc || !k_pool || !v_pool || !block_tables ||
+      !context_lens)
+    return TV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) ||
+      !aligned16(v_pool))
+    return TV_ERR_INVALID_ARG;
+  const int64_t grid_x = (int64_t)(max_query_len + 31) / 32 * num_kv_heads;
+  if (grid_x > INT32_MAX) return TV_ERR_UNSUPPORTED;
+
+  // Query rows past num_query_rows read as zeros and are never stored.
+  CUtensorMap tq, tk, tvm;
+  st = query_tensor_map(&tq, q, num_query_rows, num_q_heads,
+                        num_q_heads / num_kv_heads, 32);
+  if (st != TV_OK) return st;
+  st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TV_OK) return st;
+  st = pool_tensor_map(&tvm, v_pool, num_pages, num_kv_heads,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TV_OK) return st;
+
+  tv::PrefillArgs a{};
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.query_start_loc = query_start_loc;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.err = err;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_pages = static_cast<int>(num_pages);
+  a.max_query_len = max_query_len;
+  a.num_query_rows = num_query_rows;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return cuda_status(tv::launch_paged_prefill(
+      a, tq, tk, tvm, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal launch interface between the C ABI (tv_api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace tv {
+
+struct DecodeArgs {
+  __nv_bfloat16* out;            // [B][Hq][D]            (unsplit)
+  float* partial_out;            // [B][Hq][maxP][D]      (split)
+  float* partial_lse;            // [B][Hq][maxP]         (split)
+  const __nv_bfloat16* q;        // [B][Hq][D]
+  const int32_t* block_tables;   // [B][max_blocks_per_seq]
+  const int32_t* context_lens;   // [B]
+  uint32_t* err;                 // nullable
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int num_pages;
+  int partition_tokens;
+  int max_partitions;
+  float scale_log2;              // scale * log2(e)
+};
+
+cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
+                                const CUtensorMap& tv, int num_kv_heads,
+                                int num_seqs, int group, bool split,
+                                int parts, cudaStream_t stream);
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new,
+                             const int32_t* slot_mapping, int64_t num_tokens,
+                             void* k_pool, void* v_pool, int64_t num_slots,
+                             int row_bytes, uint32_t* err,
+                             cudaStream_t stream);
+
+cudaError_t launch_split_merge(__nv_bfloat16* out, const float* partial_out,
+                               const float* partial_lse,
+                               const int32_t* context_lens, int num_seqs,
+                               int num_q_heads, int partition_tokens,
+                               int max_partitions, cudaStream_t stream);
+
+struct PrefillArgs {
+  __nv_bfloat16* out;            // [rows][Hq][D]
+  const int32_t* query_start_loc;  // [B+1]
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  uint32_t* err;
+  int max_blocks_per_seq;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int num_pages;
+  int max_query_len;
+  int64_t num_query_rows;
+  float scale_log2;
+};
+
+cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,
+                                 const CUtensorMap& tk, const CUtensorMap& tv,
+                                 cudaStream_t stream);
+
+}  // namespace tv

@@ -16,15 +16,17 @@ Recipe (all arrays numpy; bf16 travels as uint16 bit patterns):
   * physical pages: perm = rng.permutation(num_pages); sequence s takes the
     next ceil(len_s / page_size) ids of perm, in order, as its block-table
     row; unused table entries are -1;
-  * values: K rows, then V rows, then q (then k_new, v_new) drawn as float32
-    standard normals in (sequence, position) order and rounded to bf16
-    (round to nearest even);
+  * values: float32 standard normals rounded to bf16 (nearest even), in
+    (sequence, position) order, one stream per tensor (tag 0 = cached K,
+    1 = cached V, 2 = q, 3 = k_new, 4 = v_new); chunk i of 2^22 values of
+    stream t comes from PCG64(SeedSequence(seed, spawn_key=(t, i)));
   * every pool slot that holds no cached token is bf16 NaN (0x7FC0), so a
     kernel that reads a slot it must not read produces NaN.
 """
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -52,13 +54,32 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
-def _normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
+_CHUNK = 1 << 22
+
+
+def _normal_bf16(seed: int, tag: int, shape) -> np.ndarray:
+    """bf16 N(0,1) values for stream ``tag``: chunk i of 2^22 values comes
+    from PCG64(SeedSequence(seed, spawn_key=(tag, i))), so chunks are
+    independent and are drawn on several host threads."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    step = 1 << 24
-    for i in range(0, n, step):
-        m = min(step, n - i)
-        out[i:i + m] = bf16_bits(rng.standard_normal(m, dtype=np.float32))
+
+    def fill(i):
+        g = np.random.Generator(np.random.PCG64(
+            np.random.SeedSequence(seed, spawn_key=(tag, i))))
+        lo = i * _CHUNK
+        m = min(_CHUNK, n - lo)
+        out[lo:lo + m] = bf16_bits(g.standard_normal(m, dtype=np.float32))
+
+    nchunks = -(-n // _CHUNK)
+    if nchunks <= 1:
+        for i in range(nchunks):
+            fill(i)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        workers = min(16, os.cpu_count() or 1, nchunks)
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, range(nchunks)))
     return out.reshape(shape)
 
 
@@ -184,12 +205,12 @@ def _build(name, seed, cached_lens, new_lens, num_pages, *, kind,
         seq_of = np.repeat(np.arange(b), cached)
         pos_of = np.concatenate([np.arange(c) for c in cached])
         slots = _slots(bt, seq_of, pos_of, page_size)
-        k_pool[slots] = _normal_bf16(rng, (n_cached, row))
-        v_pool[slots] = _normal_bf16(rng, (n_cached, row))
+        k_pool[slots] = _normal_bf16(seed, 0, (n_cached, row))
+        v_pool[slots] = _normal_bf16(seed, 1, (n_cached, row))
     n_new = int(new.sum())
-    q = _normal_bf16(rng, (n_new, num_q_heads, head_dim))
-    k_new = _normal_bf16(rng, (n_new, num_kv_heads, head_dim))
-    v_new = _normal_bf16(rng, (n_new, num_kv_heads, head_dim))
+    q = _normal_bf16(seed, 2, (n_new, num_q_heads, head_dim))
+    k_new = _normal_bf16(seed, 3, (n_new, num_kv_heads, head_dim))
+    v_new = _normal_bf16(seed, 4, (n_new, num_kv_heads, head_dim))
     if n_new:
         seq_of = np.repeat(np.arange(b), new)
         pos_of = np.concatenate(

@@ -1,0 +1,107 @@
+"""The C-ABI library loads and exports every symbol include/tv.h declares,
+and host-side argument checks reject bad calls before anything is launched.
+None of these tests needs a GPU: every call here returns before CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_376_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(tv_\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    names = _declared()
+    assert {"tv_kv_append", "tv_paged_decode", "tv_paged_decode_split",
+            "tv_split_merge", "tv_paged_prefill"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert names == set(_lib.SIGNATURES), names ^ set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.tv_status_string(0) == b"TV_OK"
+    assert lib.tv_status_string(2) == b"TV_ERR_UNSUPPORTED"
+    assert lib.tv_version() >= 100
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_unsupported_shapes_are_rejected_before_launch(lib):
+    p = _fake()
+    # head_dim 128
+    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 128, 16, 10,
+                               0.1, None, None) == 2
+    # page size 32
+    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 64, 32, 10,
+                               0.1, None, None) == 2
+    # 12 query heads over 8 KV heads
+    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 12, 8, 64, 16, 10,
+                               0.1, None, None) == 2
+    # GQA ratio 16
+    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 2, 64, 16, 10,
+                               0.1, None, None) == 2
+    assert lib.tv_kv_append(p, p, p, 4, p, p, 10, 8, 96, 16, None,
+                            None) == 2
+    assert lib.tv_split_merge(p, p, p, p, 2, 32, 32, 512, 4, None) == 2
+    # prefill needs 4 query heads per KV head
+    assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, 4, p, 1, 8, 8, 8, 64,
+                                16, 10, 0.1, None, None) == 2
+
+
+def test_invalid_arguments_are_rejected_before_launch(lib):
+    p = _fake()
+    unaligned = _fake(0x10008)
+    # null q
+    assert lib.tv_paged_decode(p, None, p, p, p, 4, p, 1, 32, 8, 64, 16, 10,
+                               0.1, None, None) == 1
+    # misaligned pool
+    assert lib.tv_paged_decode(p, p, unaligned, p, p, 4, p, 1, 32, 8, 64, 16,
+                               10, 0.1, None, None) == 1
+    # non-finite scale
+    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 64, 16, 10,
+                               float("nan"), None, None) == 1
+    # partition not a multiple of the page size
+    assert lib.tv_paged_decode_split(p, p, p, p, p, p, 4, p, 1, 32, 8, 64,
+                                     16, 10, 0.1, 100, 4, None, None) == 1
+    # negative token count
+    assert lib.tv_kv_append(p, p, p, -1, p, p, 10, 8, 64, 16, None,
+                            None) == 1
+    assert lib.tv_split_merge(None, p, p, p, 2, 32, 64, 512, 4, None) == 1
+
+
+def test_empty_work_is_a_no_op(lib):
+    p = _fake()
+    assert lib.tv_kv_append(None, None, None, 0, p, p, 10, 8, 64, 16, None,
+                            None) == 0
+    assert lib.tv_paged_decode(None, None, None, None, None, 4, None, 0, 32,
+                               8, 64, 16, 10, 0.1, None, None) == 0
+    assert lib.tv_paged_prefill(None, None, 0, None, None, None, None, 4,
+                                None, 0, 0, 32, 8, 64, 16, 10, 0.1, None,
+                                None) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(_lib.TVError):
+        _lib.load(str(tmp_path / "nope.so"))

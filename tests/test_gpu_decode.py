@@ -1,0 +1,142 @@
+"""Paged decode on the GPU against the oracle (elementwise parity bound)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_parity, bf16_bits, err_word, gpu_append,
+                      gpu_decode, oracle_after_append, require_gpu, upload)
+from paged_kv_cache_376_b200 import _lib
+from paged_kv_cache_376_b200 import workloads as W
+from paged_kv_cache_376_b200.workloads import bf16_bits as f32_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _run(wl):
+    """Append then decode on the GPU; oracle append then decode on the CPU."""
+    db = upload(wl)
+    gpu_append(db)
+    out = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    return db, out, ref
+
+
+def test_tiny_decode_config():
+    wl = W.tiny_decode()
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, "tiny")
+    # context 1: the output is the appended V row, bit for bit
+    v0 = np.repeat(wl.v_new[0], 4, axis=0)
+    np.testing.assert_array_equal(bf16_bits(out[0]), v0)
+    assert err_word(db) == 0
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (16, 8), (32, 4)],
+                         ids=["gqa4", "mha", "gqa2", "gqa8"])
+def test_ragged_contexts_and_group_sizes(hq, hkv):
+    lens = [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 1000,
+            4099]
+    wl = W.decode_workload(lens, num_pages=sum(-(-n // 16) for n in lens) + 7,
+                           seed=101, num_q_heads=hq, num_kv_heads=hkv)
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, f"hq={hq} hkv={hkv}")
+    assert err_word(db) == 0
+
+
+def test_llama_decode_config_full():
+    wl = W.llama_decode()
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, "llama b64 ctx2048")
+    assert err_word(db) == 0
+
+
+def test_continuous_mix_config_full():
+    wl = W.continuous_mix()
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, "mix b256")
+    assert err_word(db) == 0
+
+
+def test_empty_context_gives_zero_rows():
+    wl = W.decode_workload([3, 40], num_pages=8, seed=5)
+    db = upload(wl)
+    gpu_append(db)
+    db.context_lens[0] = 0
+    out = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    assert (out[0].float() == 0).all()
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables,
+                              np.array([0, 40], np.int32), wl.scale)
+    assert_parity(out, ref, "ctx 0")
+
+
+def test_physical_page_permutation_is_bit_identical():
+    wl = W.decode_workload([70, 513, 16, 200], num_pages=60, seed=9)
+    kp, vp = oracle_after_append(wl)
+    rng = np.random.default_rng(3)
+    perm = rng.permutation(wl.num_pages)
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm], vp2[perm] = kp, vp
+    bt2 = np.where(wl.block_tables >= 0,
+                   perm[np.maximum(wl.block_tables, 0)], -1).astype(np.int32)
+    outs = []
+    for k, v, bt in ((kp, vp, wl.block_tables), (kp2, vp2, bt2)):
+        wl.k_pool, wl.v_pool, wl.block_tables = k, v, bt
+        db = upload(wl)
+        outs.append(bf16_bits(gpu_decode(db, wl.scale)))
+    np.testing.assert_array_equal(outs[0], outs[1])
+
+
+def test_needle_dominates_at_long_context():
+    n = 20000
+    wl = W.decode_workload([n, 333], seed=11)
+    kp, vp = oracle_after_append(wl)
+    g = 3
+    q = wl.q.copy()
+    q[0, 4 * g:4 * g + 4] = q[0, 4 * g]          # same query for the group
+    needle = 12345
+    page, off = wl.block_tables[0, needle // 16], needle % 16
+    qf = W.bf16_to_f64(q[0, 4 * g]).astype(np.float32)
+    kp[page, off, g] = f32_to_bf16(qf * 8.0)     # logit ~ |q|^2 ~ 64
+    wl.q, wl.k_pool, wl.v_pool = q, kp, vp
+    db = upload(wl)
+    out = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    got = bf16_bits(out[0, 4 * g:4 * g + 4])
+    want = np.repeat(vp[page, off, g][None], 4, axis=0)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bad_page_id_is_flagged_and_left_out():
+    wl = W.decode_workload([50, 90], num_pages=12, seed=13)
+    kp, vp = oracle_after_append(wl)
+    wl.k_pool, wl.v_pool = kp, vp
+    bt = wl.block_tables.copy()
+    bt[1, 2] = wl.num_pages + 5
+    wl.block_tables = bt
+    db = upload(wl)
+    out = gpu_decode(db, wl.scale)
+    assert err_word(db) & _lib.DEVERR_BAD_PAGE
+    ref = oracle.paged_decode(wl.q, kp, vp, bt, wl.context_lens, wl.scale,
+                              allow_bad=True)
+    assert_parity(out, ref, "bad page")
+
+
+def test_context_beyond_block_table_is_clamped_and_flagged():
+    wl = W.decode_workload([40], num_pages=4, seed=17)
+    kp, vp = oracle_after_append(wl)
+    wl.k_pool, wl.v_pool = kp, vp
+    db = upload(wl)
+    db.context_lens[0] = 10_000
+    gpu_decode(db, wl.scale)
+    assert err_word(db) & _lib.DEVERR_BAD_CONTEXT

@@ -1,0 +1,112 @@
+"""Chunked prefill on the tcgen05 tensor cores against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_parity, bf16_bits, err_word, gpu_append,
+                      gpu_decode, gpu_prefill, oracle_after_append,
+                      require_gpu, upload)
+from paged_kv_cache_376_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _run(wl):
+    db = upload(wl)
+    gpu_append(db)
+    maxq = int(np.diff(wl.query_start_loc).max())
+    out = gpu_prefill(db, wl.scale, maxq)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    return db, out, kp, vp
+
+
+@pytest.mark.parametrize("prefixes,chunks", [
+    ([0], [1]),
+    ([0], [200]),
+    ([0, 5, 16, 100], [1, 31, 33, 64]),
+    ([7, 129, 1000], [95, 130, 257]),
+    ([4096, 0, 333], [32, 512, 17]),
+], ids=["one-row", "no-prefix", "ragged", "mixed", "long-prefix"])
+def test_prefill_matches_oracle_on_every_row(prefixes, chunks):
+    wl = W.prefill_workload(prefixes, chunks, seed=31)
+    db, out, kp, vp = _run(wl)
+    ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp,
+                               wl.block_tables, wl.context_lens, wl.scale)
+    assert_parity(out, ref, f"prefill {prefixes} {chunks}")
+    assert err_word(db) == 0
+
+
+def test_chunked_prefill_config_sampled():
+    wl = W.chunked_prefill()
+    db, out, kp, vp = _run(wl)
+    assert err_word(db) == 0
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(5)
+    rows = wl.q.shape[0]
+    ti = rng.integers(0, rows, 1500).astype(np.int32)
+    # always include every sequence's first and last row
+    ends = np.concatenate([wl.query_start_loc[:-1],
+                           wl.query_start_loc[1:] - 1]).astype(np.int32)
+    ti = np.concatenate([ti, ends])
+    hi = rng.integers(0, wl.num_q_heads, ti.shape[0]).astype(np.int32)
+    ref = oracle.paged_prefill_rows(wl.q, wl.query_start_loc, kp, vp,
+                                    wl.block_tables, wl.context_lens,
+                                    wl.scale, ti, hi)
+    got = out[torch.from_numpy(ti).long(), torch.from_numpy(hi).long()]
+    assert_parity(got, ref, "chunked prefill sampled")
+
+
+def test_one_row_chunk_equals_decode():
+    lens = [1, 40, 777]
+    wl = W.prefill_workload([n - 1 for n in lens], [1] * len(lens), seed=32)
+    db = upload(wl)
+    gpu_append(db)
+    a = gpu_prefill(db, wl.scale, 1)
+    b = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(a, ref, "prefill T=1")
+    assert_parity(b, ref, "decode")
+
+
+def test_rows_do_not_see_later_keys():
+    wl = W.prefill_workload([50], [100], seed=33)
+    db, out, kp, vp = _run(wl)
+    # change keys/values from position 50 + 60 on: rows 0..59 must not move
+    cut = 50 + 60
+    for j in range(cut, 150):
+        page, off = wl.block_tables[0, j // 16], j % 16
+        kp[page, off] = 0x3F80
+        vp[page, off] = 0x4000
+    wl.k_pool, wl.v_pool = kp, vp
+    db2 = upload(wl)
+    out2 = gpu_prefill(db2, wl.scale, 100)
+    torch.cuda.synchronize()
+    a, b = bf16_bits(out), bf16_bits(out2)
+    np.testing.assert_array_equal(a[:60], b[:60])
+    assert not np.array_equal(a[60:], b[60:])
+
+
+def test_physical_page_permutation_is_bit_identical():
+    wl = W.prefill_workload([300, 20], [70, 33], num_pages=80, seed=34)
+    kp, vp = oracle_after_append(wl)
+    perm = np.random.default_rng(6).permutation(wl.num_pages)
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm], vp2[perm] = kp, vp
+    bt2 = np.where(wl.block_tables >= 0,
+                   perm[np.maximum(wl.block_tables, 0)], -1).astype(np.int32)
+    outs = []
+    for k, v, bt in ((kp, vp, wl.block_tables), (kp2, vp2, bt2)):
+        wl.k_pool, wl.v_pool, wl.block_tables = k, v, bt
+        db = upload(wl)
+        outs.append(bf16_bits(gpu_prefill(db, wl.scale, 70)))
+    np.testing.assert_array_equal(outs[0], outs[1])

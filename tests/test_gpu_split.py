@@ -1,0 +1,123 @@
+"""Split-KV decode partials and their log-sum-exp merge on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_parity, bf16_bits, err_word, gpu_append,
+                      gpu_decode, gpu_merge, gpu_split, oracle_after_append,
+                      require_gpu, to_f64, upload)
+from paged_kv_cache_376_b200 import workloads as W
+from paged_kv_cache_376_b200.workloads import bf16_bits as f32_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _lse_close(gpu, ref, what):
+    g = to_f64(gpu)
+    fin = np.isfinite(ref)
+    assert (np.isneginf(g) == ~fin).all(), f"{what}: empty partitions differ"
+    np.testing.assert_allclose(g[fin], ref[fin], rtol=1e-5, atol=1e-4,
+                               err_msg=what)
+
+
+@pytest.mark.parametrize("pt", [16, 512])
+def test_partials_match_oracle(pt):
+    lens = [1, 17, 511, 512, 513, 1500, 3000]
+    wl = W.decode_workload(lens, seed=21)
+    maxp = -(-max(lens) // pt) + 1          # one always-empty partition
+    db = upload(wl)
+    gpu_append(db)
+    po, pl = gpu_split(db, wl.scale, pt, maxp)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ro, rl = oracle.paged_decode_partials(wl.q, kp, vp, wl.block_tables,
+                                          wl.context_lens, wl.scale, pt, maxp)
+    assert_parity(po, ro, f"o_p pt={pt}")
+    _lse_close(pl, rl, f"lse_p pt={pt}")
+    assert err_word(db) == 0
+
+
+def test_merge_kernel_matches_oracle_merge_on_the_same_partials():
+    wl = W.decode_workload([100, 2000, 4097], seed=22)
+    kp, vp = oracle_after_append(wl)
+    pt = 512
+    maxp = 10
+    ro, rl = oracle.paged_decode_partials(wl.q, kp, vp, wl.block_tables,
+                                          wl.context_lens, wl.scale, pt, maxp)
+    ro32, rl32 = ro.astype(np.float32), rl.astype(np.float32)
+    db = upload(wl)
+    out = gpu_merge(db, torch.from_numpy(ro32).cuda(),
+                    torch.from_numpy(rl32).cuda(), pt)
+    ref = oracle.split_merge(ro32.astype(np.float64), rl32.astype(np.float64),
+                             wl.context_lens, pt)
+    assert_parity(out, ref, "merge")
+
+
+def test_split_then_merge_matches_decode_oracle():
+    lens = [1, 600, 5000, 9999]
+    wl = W.decode_workload(lens, seed=23)
+    pt = 512
+    maxp = -(-max(lens) // pt)
+    db = upload(wl)
+    gpu_append(db)
+    po, pl = gpu_split(db, wl.scale, pt, maxp)
+    out = gpu_merge(db, po, pl, pt)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, "split+merge")
+
+
+def test_one_partition_equals_unsplit_decode_bitwise():
+    lens = [3, 77, 480, 512]
+    wl = W.decode_workload(lens, seed=24)
+    db = upload(wl)
+    gpu_append(db)
+    po, pl = gpu_split(db, wl.scale, 512, 1)
+    merged = gpu_merge(db, po, pl, 512)
+    direct = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bf16_bits(merged), bf16_bits(direct))
+
+
+def test_long_split_config_sampled_rows_and_needles():
+    wl = W.long_split()
+    pt = wl.partition_tokens
+    maxp = wl.max_partitions()
+    kp, vp = oracle_after_append(wl)
+    # needles: sequence 1 head group 2 at the first, a middle and the last
+    # partition, and at a page's last slot; each needle query group shares q
+    q = wl.q.copy()
+    needles = {1: 5, 3: 131072 // 2 + 77, 5: 131071 - 3, 6: 16 * 4000 + 15}
+    for s, pos in needles.items():
+        g = 2
+        q[s, 4 * g:4 * g + 4] = q[s, 4 * g]
+        page, off = wl.block_tables[s, pos // 16], pos % 16
+        qf = W.bf16_to_f64(q[s, 4 * g]).astype(np.float32)
+        kp[page, off, g] = f32_to_bf16(qf * 8.0)
+    wl.q, wl.k_pool, wl.v_pool = q, kp, vp
+    db = upload(wl)
+    po, pl = gpu_split(db, wl.scale, pt, maxp)
+    out = gpu_merge(db, po, pl, pt)
+    torch.cuda.synchronize()
+    assert err_word(db) == 0
+    rng = np.random.default_rng(4)
+    si = rng.integers(0, wl.num_seqs, 12).astype(np.int32)
+    hi = rng.integers(0, wl.num_q_heads, 12).astype(np.int32)
+    ref = oracle.paged_decode_rows(wl.q, kp, vp, wl.block_tables,
+                                   wl.context_lens, wl.scale, si, hi)
+    assert_parity(out[torch.from_numpy(si).long(),
+                      torch.from_numpy(hi).long()], ref, "long sampled")
+    for s, pos in needles.items():
+        page, off = wl.block_tables[s, pos // 16], pos % 16
+        got = bf16_bits(out[s, 8:12])
+        np.testing.assert_array_equal(got, np.repeat(vp[page, off, 2][None],
+                                                     4, axis=0))
+    assert torch.isfinite(out.float()).all()
