@@ -101,27 +101,32 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   __syncwarp();
 
   // ---- q for the G heads of this KV head, pre-scaled by scale*log2(e) -----
-  float qf[G][8];
+  // Element pairs (2i, 2i+1) of this lane's 8-element chunk, as float2 so
+  // the dot products run on the packed fp32x2 FMA pipe.
+  float2 q2[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const uint4 v = *reinterpret_cast<const uint4*>(
         a.q + ((size_t)seq * a.num_q_heads + kvh * G + h) * kD + chk * 8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      qf[h][2 * i] = bf16_lo(w[i]) * a.scale_log2;
-      qf[h][2 * i + 1] = bf16_hi(w[i]) * a.scale_log2;
-    }
+    for (int i = 0; i < 4; ++i)
+      q2[h][i] = make_float2(bf16_lo(w[i]) * a.scale_log2,
+                             bf16_hi(w[i]) * a.scale_log2);
   }
 
-  float m_run[G], l_run[G], acc[G][8];
+  // After the reduce-scatter below, lane chunk c holds the score of head
+  // c >> kShift (lanes that share a head hold the same value); head h is
+  // read from lane (group, h << kShift).
+  constexpr int kShift = G == 8 ? 0 : G == 4 ? 1 : G == 2 ? 2 : 3;
+  const int my_head = chk >> kShift;
+
+  float m_run = -INFINITY, l_run = 0.f;   // for head my_head
+  float2 acc2[G][4];                      // all heads, this lane's 8 dims
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m_run[h] = -INFINITY;
-    l_run[h] = 0.f;
+  for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-  }
+    for (int i = 0; i < 4; ++i) acc2[h][i] = make_float2(0.f, 0.f);
 
   // Block-table entries of this warp's pages, 32 per batch, one per lane.
   auto load_pids = [&](int batch) -> int {
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   int pid_next = load_pids(1);
   const uint64_t policy = l2_policy_evict_first();
 
-  auto issue = [&](int i, int pid, int stage) {
+  auto issue = [&](int pid, int stage) {
     const bool ok = pid >= 0 && pid < a.num_pages;
     if (!ok) flag_error(a.err, DEVERR_BAD_PAGE);
     const int y = (ok ? pid : 0) * kPS;
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 #pragma unroll
   for (int j = 0; j < kStages; ++j) {
     const int pid = __shfl_sync(0xffffffffu, pid_cur, j);
-    if (lane == 0 && j < my_n) issue(j, pid, j);
+    if (lane == 0 && j < my_n) issue(pid, j);
   }
 
   bool failed = false;
@@ -163,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     const int pid = __shfl_sync(0xffffffffu, pid_cur, i & 31);
     const bool page_ok = pid >= 0 && pid < a.num_pages;
     const int page_tok0 = (first_page + warp + kWarps * i) * kPS;
+    // warp-uniform: every token of the page is a real key of this range
+    const bool full_page = page_ok && page_tok0 + kPS <= tok_end;
 
     // Every lane observes the barrier (acquire of the TMA bytes); the
     // outcome is made warp-uniform so the warp never diverges on it.
@@ -174,86 +181,105 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     const uint8_t* kbase = &sm.ring[warp][stage][0];
     const uint8_t* vbase = kbase + kSliceBytes;
 
-    // ---- scores for the 4 tokens of this lane group ------------------------
-    float s[4][G];
+    // ---- scores: token it*4+grp, head my_head ---------------------------------
+    float s[4];
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int r = it * 4 + grp;
       const uint4 kv =
           *reinterpret_cast<const uint4*>(kbase + r * kRowBytes + chk * 16);
       const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-      float kf[8];
+      float2 k2[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        kf[2 * t] = bf16_lo(w[t]);
-        kf[2 * t + 1] = bf16_hi(w[t]);
-      }
+      for (int t = 0; t < 4; ++t) k2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
+      float part[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float d = 0.f;
+        float2 d2 = __fmul2_rn(q2[h][0], k2[0]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(qf[h][e], kf[e], d);
-        s[it][h] = d;
+        for (int t = 1; t < 4; ++t) d2 = __ffma2_rn(q2[h][t], k2[t], d2);
+        part[h] = d2.x + d2.y;
       }
+      // reduce-scatter over the 8 lanes of the group: at each xor step a
+      // lane keeps half of its values and adds the partner's copy of them
+      int n = G;
 #pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
+      for (int off = 4; off >= 1; off >>= 1) {
+        if (n > 1) {
+          const bool upper = (chk & off) != 0;
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          s[it][h] += __shfl_xor_sync(0xffffffffu, s[it][h], off);
+          for (int h = 0; h < G / 2; ++h) {
+            if (h < n / 2) {
+              const float keep = upper ? part[h + n / 2] : part[h];
+              const float send = upper ? part[h] : part[h + n / 2];
+              part[h] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+          }
+          n >>= 1;
+        } else {
+          part[0] += __shfl_xor_sync(0xffffffffu, part[0], off);
+        }
       }
-      const bool valid = page_ok && (page_tok0 + r) < tok_end;
-#pragma unroll
-      for (int h = 0; h < G; ++h) s[it][h] = valid ? s[it][h] : -INFINITY;
+      s[it] = part[0];
+      if (!full_page) {
+        const bool valid = page_ok && (page_tok0 + r) < tok_end;
+        s[it] = valid ? s[it] : -INFINITY;
+      }
     }
 
-    // ---- online softmax, once per page -------------------------------------
-    float alpha[G], m_use[G];
+    // ---- online softmax, once per page -----------------------------------------
+    float pm = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
+    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
+    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
+    if (__any_sync(0xffffffffu, pm > m_run)) {
+      // the running max moved for some head: rescale (rare after warm-up)
+      const float m_new = fmaxf(m_run, pm);
+      const float alpha = fast_exp2(m_run - (m_new == -INFINITY ? 0.f : m_new));
+      m_run = m_new;
+      l_run *= alpha;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float pm = fmaxf(fmaxf(s[0][h], s[1][h]), fmaxf(s[2][h], s[3][h]));
-      pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
-      pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
-      const float m_new = fmaxf(m_run[h], pm);
-      m_use[h] = m_new == -INFINITY ? 0.f : m_new;
-      alpha[h] = fast_exp2(m_run[h] - m_use[h]);
-      m_run[h] = m_new;
-      l_run[h] *= alpha[h];
+      for (int h = 0; h < G; ++h) {
+        const float ah = __shfl_sync(0xffffffffu, alpha, h << kShift);
+        const float2 a2 = make_float2(ah, ah);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] *= alpha[h];
+        for (int t = 0; t < 4; ++t) acc2[h][t] = __fmul2_rn(acc2[h][t], a2);
+      }
     }
+    const float m_use = m_run == -INFINITY ? 0.f : m_run;
 
-    // ---- P.V ----------------------------------------------------------------
+    // ---- P.V -------------------------------------------------------------------
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int r = it * 4 + grp;
-      const bool valid = page_ok && (page_tok0 + r) < tok_end;
+      const float p = fast_exp2(s[it] - m_use);
+      l_run += p;
       uint4 vv =
           *reinterpret_cast<const uint4*>(vbase + r * kRowBytes + chk * 16);
-      if (!valid) vv = make_uint4(0, 0, 0, 0);  // stale slots may hold NaN
-      const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-      float vf[8];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        vf[2 * t] = bf16_lo(w[t]);
-        vf[2 * t + 1] = bf16_hi(w[t]);
+      if (!full_page) {
+        const bool valid = page_ok && (page_tok0 + r) < tok_end;
+        if (!valid) vv = make_uint4(0, 0, 0, 0);  // stale slots may be NaN
       }
+      const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+      float2 v2[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) v2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float p = fast_exp2(s[it][h] - m_use[h]);
-        l_run[h] += p;
+        const float ph = __shfl_sync(0xffffffffu, p, grp * 8 + (h << kShift));
+        const float2 p2 = make_float2(ph, ph);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(p, vf[e], acc[h][e]);
+        for (int t = 0; t < 4; ++t) acc2[h][t] = __ffma2_rn(p2, v2[t], acc2[h][t]);
       }
     }
 
-    // ---- hand the slot back to the TMA unit ----------------------------------
+    // ---- hand the slot back to the TMA unit ------------------------------------
     fence_proxy_async_smem();
     __syncwarp();
     const int j = i + kStages;
     const int src = ((j >> 5) == (i >> 5)) ? pid_cur : pid_next;
     const int pid_j = __shfl_sync(0xffffffffu, src, j & 31);
     if (j < my_n) {
-      if (lane == 0) issue(j, pid_j, stage);
+      if (lane == 0) issue(pid_j, stage);
       ++issued;
     }
   }
@@ -264,37 +290,40 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     if (lane == 0) flag_error(a.err, DEVERR_TIMEOUT);
     for (int k = i; k < issued; ++k)
       mbar_wait(smem_u32(&sm.full[warp][k % kStages]), (k / kStages) & 1);
+    m_run = -INFINITY;
+    l_run = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_run[h] = -INFINITY;
-      l_run[h] = 0.f;
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-    }
+      for (int t = 0; t < 4; ++t) acc2[h][t] = make_float2(0.f, 0.f);
   }
 
-  // ---- reduce over the 4 lane groups ----------------------------------------
+  // ---- reduce over the 4 lane groups ------------------------------------------
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 8);
-      acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 16);
+    for (int t = 0; t < 4; ++t) {
+      acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 8);
+      acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 8);
+      acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 16);
+      acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 16);
     }
   }
   __syncthreads();  // every warp is done with its ring
   auto& cb = *reinterpret_cast<Combine<G>*>(smem_raw);
   if (grp == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) cb.acc[warp][h][chk * 8 + e] = acc[h][e];
-      if (chk == 0) {
-        cb.m[warp][h] = m_run[h];
-        cb.l[warp][h] = l_run[h];
+      for (int t = 0; t < 4; ++t) {
+        cb.acc[warp][h][chk * 8 + 2 * t] = acc2[h][t].x;
+        cb.acc[warp][h][chk * 8 + 2 * t + 1] = acc2[h][t].y;
       }
+    if ((chk & ((1 << kShift) - 1)) == 0) {
+      cb.m[warp][my_head] = m_run;
+      cb.l[warp][my_head] = l_run;
     }
   }
   __syncthreads();

@@ -22,8 +22,13 @@
 //  * warp 0: TMA producer (q once, K/V through a 3-stage ring).
 //    warp 1: tensor-memory allocation and the single MMA-issuing thread:
 //      S_j = Q K_j^T (M128 N128 K16 x4) into one of two S buffers in tensor
-//      memory, then O_{j-1} = P_{j-1} V_{j-1} (M128 N64 K16 x8; V read as an
-//      MN-major operand) into one of two O buffers.
+//      memory, then O_{j-1} = P_{j-1} V_{j-1} (M128 N64 K16 x8, twice: once
+//      for P_hi and once for P_lo; V read as an MN-major operand) into one of
+//      two O buffers.
+//  * P is split as P_hi = bf16(p), P_lo = bf16(p - P_hi) so the PV product
+//    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
+//    operands); a single bf16 P carries 8 bits, which is not enough for rows
+//    that see few keys.
 //    warps 2-5: softmax.  Thread = one MMA row = one (query, head).  It reads
 //      its 128 scores with tcgen05.ld, masks causally, updates the running
 //      max/sum in base 2 (no cross-thread reduction at all), writes P as bf16
@@ -43,7 +48,7 @@ constexpr int kQRows = 32;               // query rows per CTA
 constexpr int kBM = kQRows * kG;         // 128 MMA rows
 constexpr int kBN = 128;                 // keys per tile
 constexpr int kPagesPerTile = kBN / kPS; // 8
-constexpr int kST = 3;                   // K/V ring depth
+constexpr int kST = 2;                   // K/V ring depth
 constexpr int kRowBytes = kD * 2;        // 128
 constexpr int kTileBytes = kBN * kRowBytes;  // 16 KB
 constexpr int kPageBytes = kPS * kRowBytes;  // 2 KB
@@ -57,9 +62,10 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct PrefillSmem {
   alignas(1024) uint8_t q[kBM * kRowBytes];          // 16 KB
-  alignas(1024) uint8_t k[kST][kTileBytes];          // 48 KB
-  alignas(1024) uint8_t v[kST][kTileBytes];          // 48 KB
-  alignas(1024) uint8_t p[2][2][kBM * kRowBytes];    // 64 KB: [buf][key half]
+  alignas(1024) uint8_t k[kST][kTileBytes];          // 32 KB
+  alignas(1024) uint8_t v[kST][kTileBytes];          // 32 KB
+  // P = P_hi + P_lo, both bf16: [buffer][hi/lo][key half][128 rows x 128 B]
+  alignas(1024) uint8_t p[2][2][2][kBM * kRowBytes];  // 128 KB
   alignas(8) uint64_t q_full;
   uint64_t kv_full[kST], kv_empty[kST];
   uint64_t s_full[2], s_free[2], p_full[2], o_full[2], o_free[2];
@@ -185,17 +191,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             !mbar_wait(smem_u32(&sm.o_free[b]), ((t >> 1) + 1) & 1))
           return false;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sm.p[b][0]);
         const uint32_t v_addr = smem_u32(sm.v[st]);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          // A = P: K-major, keys [16k, 16k+16) live in half k/4 at byte 32*(k%4)
-          const uint64_t ad = smem_desc_sw128(
-              p_addr + (k >> 2) * (kBM * kRowBytes) + (k & 3) * 32, 16, 1024);
-          // B = V: MN-major (head dim contiguous), 16 keys = 2 groups of 8 rows
-          const uint64_t bd =
-              smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
-          tc_mma_bf16(tmem + kOCol + b * kD, ad, bd, kIdescPV, k > 0);
+        for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
+          const uint32_t p_addr = smem_u32(sm.p[b][part][0]);
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            // A = P: K-major; keys [16k, 16k+16) sit in half k/4, byte 32*(k%4)
+            const uint64_t ad = smem_desc_sw128(
+                p_addr + (k >> 2) * (kBM * kRowBytes) + (k & 3) * 32, 16,
+                1024);
+            // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
+            const uint64_t bd =
+                smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
+            tc_mma_bf16(tmem + kOCol + b * kD, ad, bd, kIdescPV,
+                        (part | k) != 0);
+          }
         }
         tc_commit(smem_u32(&sm.o_full[b]));
         tc_commit(smem_u32(&sm.kv_empty[st]));
@@ -322,21 +333,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- P (bf16) into the swizzled K-major layout ---------------------------
+      // ---- P_hi, P_lo (bf16) into the swizzled K-major layout -------------------
       {
-        uint8_t* prow = sm.p[b][0] + r * kRowBytes;
+        uint8_t* phi = sm.p[b][0][0] + r * kRowBytes;
+        uint8_t* plo = sm.p[b][1][0] + r * kRowBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const int x = half * 64 + ch * 8;
-            uint4 w;
-            w.x = pack_bf16x2(s[x + 0], s[x + 1]);
-            w.y = pack_bf16x2(s[x + 2], s[x + 3]);
-            w.z = pack_bf16x2(s[x + 4], s[x + 5]);
-            w.w = pack_bf16x2(s[x + 6], s[x + 7]);
-            *reinterpret_cast<uint4*>(prow + half * (kBM * kRowBytes) +
-                                      ((ch ^ (r & 7)) * 16)) = w;
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi[e] = pack_bf16x2(s[x + 2 * e], s[x + 2 * e + 1]);
+              lo[e] = pack_bf16x2(s[x + 2 * e] - bf16_lo(hi[e]),
+                                  s[x + 2 * e + 1] - bf16_hi(hi[e]));
+            }
+            const int off = half * (kBM * kRowBytes) + ((ch ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(phi + off) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(plo + off) =
+                make_uint4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
       }
