@@ -10,30 +10,35 @@
 // online softmax, tile sized to on-chip memory ("Tiny-vLLM 实战：用 C++/CUDA
 // 手写高性能 LLM 推理引擎", sec. "算子融合", FlashAttention-like blocking).
 //
-// B200 design (one CTA per (KV head, 32-query tile, sequence); 6 warps):
-//  * M = 128 MMA rows = 32 query rows x the 4 query heads of one KV head, so
-//    every K/V tile feeds 4 heads (GQA reuse) and one tcgen05.mma of M = 128
-//    covers them.  q arrives by one 3-D TMA box {64 d, 4 heads, 32 rows}.
+// B200 design (one CTA per (KV head, 64-query block, sequence); 12 warps):
+//  * An MMA tile has M = 128 rows = 32 query rows x the 4 query heads of one
+//    KV head, so every K/V tile feeds 4 heads (GQA reuse).  A CTA owns two
+//    such query tiles (A: rows q0..q0+31, B: q0+32..q0+63) that share every
+//    K/V tile, and the tensor core alternates between them while the other
+//    tile's softmax runs.  q arrives by one 3-D TMA box {64 d, 4 heads, 32
+//    rows} per tile.
 //  * Keys come in tiles of 128 = 8 pages; each page of one KV head (16 rows x
 //    128 B) is one 2-D TMA box, 128-byte swizzled, so 8 boxes at 2 KB
 //    offsets form exactly the canonical K-major SW128 operand.  Pages past
 //    the range (or with a bad id) are read at an out-of-range coordinate and
 //    arrive as zeros.
-//  * warp 0: TMA producer (q once, K/V through a 3-stage ring).
+//  * warp 0: TMA producer (q once, K/V through a 2-stage ring).
 //    warp 1: tensor-memory allocation and the single MMA-issuing thread:
-//      S_j = Q K_j^T (M128 N128 K16 x4) into one of two S buffers in tensor
-//      memory, then O_{j-1} = P_{j-1} V_{j-1} (M128 N64 K16 x8, twice: once
-//      for P_hi and once for P_lo; V read as an MN-major operand) into one of
-//      two O buffers.
+//      S_t = Q_t K_j^T (M128 N128 K16 x4) into tile t's S columns, then
+//      O_t += P_t V_j (M128 N64 K16 x8, once for P_hi and once for P_lo;
+//      V read as an MN-major operand) accumulated in tile t's O columns.
+//    warps 4-7 / 8-11: softmax of tile A / B.  Thread = one MMA row = one
+//      (query, head).  Pass 1 reads its 128 scores from tensor memory and
+//      takes their maximum; the running maximum moves only when it grows by
+//      more than 2^8 (then O and l are rescaled in place, which is rare), so
+//      O stays in tensor memory across key tiles.  Pass 2 re-reads the
+//      scores, exponentiates, sums, and writes P into the swizzled K-major
+//      layout the MMA reads.  The causal mask is applied only to the tiles
+//      that cross the diagonal.
 //  * P is split as P_hi = bf16(p), P_lo = bf16(p - P_hi) so the PV product
 //    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
 //    operands); a single bf16 P carries 8 bits, which is not enough for rows
 //    that see few keys.
-//    warps 2-5: softmax.  Thread = one MMA row = one (query, head).  It reads
-//      its 128 scores with tcgen05.ld, masks causally, updates the running
-//      max/sum in base 2 (no cross-thread reduction at all), writes P as bf16
-//      into the swizzled K-major layout the MMA reads, and folds the previous
-//      tile's O into fp32 registers (o = o * alpha + O).
 //  * Every wait is an mbarrier wait bounded by a 2 s time limit.
 #include "tv_device.cuh"
 #include "tv_kernels.h"
@@ -44,7 +49,8 @@ namespace {
 constexpr int kD = 64;
 constexpr int kPS = 16;
 constexpr int kG = 4;                    // query heads per KV head
-constexpr int kQRows = 32;               // query rows per CTA
+constexpr int kQRows = 32;               // query rows per MMA tile
+constexpr int kQTiles = 2;               // MMA tiles per CTA (A, B)
 constexpr int kBM = kQRows * kG;         // 128 MMA rows
 constexpr int kBN = 128;                 // keys per tile
 constexpr int kPagesPerTile = kBN / kPS; // 8
@@ -52,23 +58,25 @@ constexpr int kST = 2;                   // K/V ring depth
 constexpr int kRowBytes = kD * 2;        // 128
 constexpr int kTileBytes = kBN * kRowBytes;  // 16 KB
 constexpr int kPageBytes = kPS * kRowBytes;  // 2 KB
-constexpr int kThreads = 192;
+constexpr int kHalfBytes = kBM * kRowBytes;  // one 64-key half of P: 16 KB
+constexpr int kThreads = 384;
 constexpr int kTmemCols = 512;
-constexpr int kSCol = 0;                 // S buffers: columns [0, 256)
-constexpr int kOCol = 2 * kBN;           // O buffers: columns [256, 384)
+constexpr int kSCol = 0;                 // S of tile t: columns [128t, 128t+128)
+constexpr int kOCol = kQTiles * kBN;     // O of tile t: [256 + 64t, +64)
+constexpr float kRescaleThreshold = 8.f; // log2 units: rescale when max grows > 2^8
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct PrefillSmem {
-  alignas(1024) uint8_t q[kBM * kRowBytes];          // 16 KB
-  alignas(1024) uint8_t k[kST][kTileBytes];          // 32 KB
-  alignas(1024) uint8_t v[kST][kTileBytes];          // 32 KB
-  // P = P_hi + P_lo, both bf16: [buffer][hi/lo][key half][128 rows x 128 B]
-  alignas(1024) uint8_t p[2][2][2][kBM * kRowBytes];  // 128 KB
+  alignas(1024) uint8_t q[kQTiles][kBM * kRowBytes];        // 32 KB
+  alignas(1024) uint8_t k[kST][kTileBytes];                 // 32 KB
+  alignas(1024) uint8_t v[kST][kTileBytes];                 // 32 KB
+  // P = P_hi + P_lo, both bf16: [tile][hi/lo][key half][128 rows x 128 B]
+  alignas(1024) uint8_t p[kQTiles][2][2][kHalfBytes];       // 128 KB
   alignas(8) uint64_t q_full;
   uint64_t kv_full[kST], kv_empty[kST];
-  uint64_t s_full[2], s_free[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[kQTiles], s_free[kQTiles], p_full[kQTiles], o_full[kQTiles];
   uint32_t tmem_base;
   uint32_t bad_pages[kST];
 };
@@ -83,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto& sm = *reinterpret_cast<PrefillSmem*>(base);
 
   const int kvh = blockIdx.x;
-  const int tile = gridDim.y - 1 - blockIdx.y;   // heaviest tiles first
+  const int blk = gridDim.y - 1 - blockIdx.y;    // heaviest blocks first
   const int seq = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -93,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int T = a.query_start_loc[seq + 1] - qs;
   int ctx = a.context_lens[seq];
   const int ctx_cap = a.max_blocks_per_seq * kPS;
-  const int q0 = tile * kQRows;
+  const int q0 = blk * kQRows * kQTiles;
   if (q0 >= T) return;
   if (ctx > ctx_cap) {
     if (threadIdx.x == 0) flag_error(a.err, DEVERR_BAD_CONTEXT);
@@ -104,9 +112,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   const int P = ctx - T;                      // cached prefix length
-  const int q_hi = min(q0 + kQRows, T);       // rows [q0, q_hi) are real
-  const int n_keys = P + q_hi;                // keys [0, n_keys) are needed
-  const int n_tiles = (n_keys + kBN - 1) / kBN;
+  // tile t covers query rows [q0 + 32t, q0 + 32t + 32) of the chunk
+  int n_tiles_of[kQTiles];
+#pragma unroll
+  for (int t = 0; t < kQTiles; ++t) {
+    const int lo = q0 + t * kQRows;
+    const int hi = min(lo + kQRows, T);
+    n_tiles_of[t] = hi > lo ? (P + hi + kBN - 1) / kBN : 0;
+  }
+  const int n_tiles = max(n_tiles_of[0], n_tiles_of[1]);
+  const int n_keys = P + min(q0 + kQRows * kQTiles, T);   // keys loaded
   const int n_pages = (n_keys + kPS - 1) / kPS;
   const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
 
@@ -117,12 +132,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.kv_full[i]), 1);
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_free[i]), 4);
-      mbar_init(smem_u32(&sm.p_full[i]), 4);
-      mbar_init(smem_u32(&sm.o_full[i]), 1);
-      mbar_init(smem_u32(&sm.o_free[i]), 4);
+    for (int t = 0; t < kQTiles; ++t) {
+      mbar_init(smem_u32(&sm.s_full[t]), 1);
+      mbar_init(smem_u32(&sm.s_free[t]), 4);
+      mbar_init(smem_u32(&sm.p_full[t]), 4);
+      mbar_init(smem_u32(&sm.o_full[t]), 1);
     }
     fence_mbar_init();
   }
@@ -139,8 +153,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= TMA producer =====================================
     if (lane == 0) {
       const uint32_t qbar = smem_u32(&sm.q_full);
-      mbar_arrive_expect_tx(qbar, kBM * kRowBytes);
-      tma_load_3d(smem_u32(sm.q), &tm_q, 0, kvh * kG, qs + q0, qbar);
+      mbar_arrive_expect_tx(qbar, kQTiles * kBM * kRowBytes);
+#pragma unroll
+      for (int t = 0; t < kQTiles; ++t)
+        tma_load_3d(smem_u32(sm.q[t]), &tm_q, 0, kvh * kG,
+                    qs + q0 + t * kQRows, qbar);
       const int oob_row = a.num_pages * kPS;   // reads as zeros
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j % kST;
@@ -182,205 +199,219 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= MMA issuer =======================================
     if (lane == 0) {
       bool ok = mbar_wait(smem_u32(&sm.q_full), 0);
-      const uint32_t q_addr = smem_u32(sm.q);
-      auto issue_pv = [&](int t) -> bool {
-        const int b = t & 1;
-        const int st = t % kST;
-        if (!mbar_wait(smem_u32(&sm.p_full[b]), (t >> 1) & 1)) return false;
-        if (t >= 2 &&
-            !mbar_wait(smem_u32(&sm.o_free[b]), ((t >> 1) + 1) & 1))
+      auto issue_qk = [&](int t, int j) -> bool {
+        if (j >= 1 && !mbar_wait(smem_u32(&sm.s_free[t]), (j - 1) & 1))
           return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.v[st]);
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
-          const uint32_t p_addr = smem_u32(sm.p[b][part][0]);
-#pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            // A = P: K-major; keys [16k, 16k+16) sit in half k/4, byte 32*(k%4)
-            const uint64_t ad = smem_desc_sw128(
-                p_addr + (k >> 2) * (kBM * kRowBytes) + (k & 3) * 32, 16,
-                1024);
-            // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
-            const uint64_t bd =
-                smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
-            tc_mma_bf16(tmem + kOCol + b * kD, ad, bd, kIdescPV,
-                        (part | k) != 0);
-          }
-        }
-        tc_commit(smem_u32(&sm.o_full[b]));
-        tc_commit(smem_u32(&sm.kv_empty[st]));
-        return true;
-      };
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % kST;
-        const int b = j & 1;
-        if (!mbar_wait(smem_u32(&sm.kv_full[st]), (j / kST) & 1) ||
-            (j >= 2 &&
-             !mbar_wait(smem_u32(&sm.s_free[b]), ((j >> 1) + 1) & 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.k[st]);
+        const uint32_t q_addr = smem_u32(sm.q[t]);
+        const uint32_t k_addr = smem_u32(sm.k[j % kST]);
 #pragma unroll
         for (int k = 0; k < kD / 16; ++k) {
           const uint64_t ad = smem_desc_sw128(q_addr + k * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_addr + k * 32, 16, 1024);
-          tc_mma_bf16(tmem + kSCol + b * kBN, ad, bd, kIdescQK, k > 0);
+          tc_mma_bf16(tmem + kSCol + t * kBN, ad, bd, kIdescQK, k > 0);
         }
-        tc_commit(smem_u32(&sm.s_full[b]));
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+        tc_commit(smem_u32(&sm.s_full[t]));
+        return true;
+      };
+      auto issue_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait(smem_u32(&sm.p_full[t]), j & 1)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sm.v[j % kST]);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
+          const uint32_t p_addr = smem_u32(sm.p[t][part][0]);
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            // A = P: K-major; keys [16k, 16k+16) sit in half k/4, byte 32*(k%4)
+            const uint64_t ad = smem_desc_sw128(
+                p_addr + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 1024);
+            // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
+            const uint64_t bd =
+                smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
+            tc_mma_bf16(tmem + kOCol + t * kD, ad, bd, kIdescPV,
+                        (j | part | k) != 0);
+          }
         }
+        tc_commit(smem_u32(&sm.o_full[t]));
+        return true;
+      };
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        if (j < n_tiles) {
+          if (!mbar_wait(smem_u32(&sm.kv_full[j % kST]), (j / kST) & 1)) {
+            ok = false;
+            break;
+          }
+        }
+        // S for tile j, P.V for tile j - 1, interleaving the two query tiles
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+          if (ok && j < n_tiles_of[t] && !issue_qk(t, j)) ok = false;
+          if (ok && j >= 1 && j - 1 < n_tiles_of[t] && !issue_pv(t, j - 1))
+            ok = false;
+        }
+        if (!ok) break;
+        if (j >= 1) tc_commit(smem_u32(&sm.kv_empty[(j - 1) % kST]));
       }
-      if (ok && !issue_pv(n_tiles - 1)) ok = false;
       if (!ok) flag_error(a.err, DEVERR_TIMEOUT);
     }
-  } else {
-    // ======================= softmax warps ====================================
+  } else if (warp >= 4) {
+    // ======================= softmax warpgroups ===============================
+    const int t = (warp >> 2) - 1;           // query tile: 0 = A, 1 = B
     const int quarter = warp & 3;            // tensor-memory lane quarter
     const int r = quarter * 32 + lane;       // MMA row
+    const int qt0 = q0 + t * kQRows;         // first chunk row of this tile
     const int qi = r >> 2;                   // query row within the tile
     const int hh = r & 3;                    // head within the group
-    const bool row_real = q0 + qi < T;
-    const int limit = row_real ? P + q0 + qi : ctx - 1;  // last visible key
+    const bool row_real = qt0 + qi < T;
+    const int limit = row_real ? P + qt0 + qi : ctx - 1;  // last visible key
+    const int my_tiles = n_tiles_of[t];
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + kSCol + t * kBN;
+    const uint32_t o_addr = tmem + lane_base + kOCol + t * kD;
     const float c = a.scale_log2;
 
-    float o[kD];
-#pragma unroll
-    for (int d = 0; d < kD; ++d) o[d] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 1.f;
+    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-
-    auto fold_o = [&](int t, float alpha) -> bool {
-      const int b = t & 1;
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(smem_u32(&sm.o_full[b]), (t >> 1) & 1)))
-        return false;
-      tc_fence_after();
-      float ov[32];
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        tmem_ld32(tmem + lane_base + kOCol + b * kD + h2 * 32, ov);
-#pragma unroll
-        for (int d = 0; d < 32; ++d)
-          o[h2 * 32 + d] = fmaf(o[h2 * 32 + d], alpha, ov[d]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.o_free[b]));
-      return true;
-    };
-
-    for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
+    for (int j = 0; j < my_tiles; ++j) {
       const int st = j % kST;
+      const int key0 = j * kBN;
+      // every row of the tile sees every key of key tile j?
+      const bool full_tile = key0 + kBN - 1 <= P + qt0;
       if (!__all_sync(0xffffffffu,
-                      mbar_wait(smem_u32(&sm.s_full[b]), (j >> 1) & 1))) {
+                      mbar_wait(smem_u32(&sm.s_full[t]), j & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int cq = 0; cq < kBN / 32; ++cq) {
-        float tmp[32];
-        tmem_ld32(tmem + lane_base + kSCol + b * kBN + cq * 32, tmp);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[cq * 32 + x] = tmp[x];
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[b]));
-
-      // ---- mask, running max, exponentials --------------------------------
-      const int key0 = j * kBN;
       const uint32_t bad = sm.bad_pages[st];
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < kBN; ++x) {
-        const int key = key0 + x;
-        const bool vis = key <= limit && !((bad >> (x / kPS)) & 1u);
-        s[x] = vis ? s[x] * c : -INFINITY;
-        tmax = fmaxf(tmax, s[x]);
-      }
-      const float m_new = fmaxf(m_run, tmax);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = fast_exp2(m_run - m_use);
-      float lsum = 0.f;
-#pragma unroll
-      for (int x = 0; x < kBN; ++x) {
-        s[x] = fast_exp2(s[x] - m_use);
-        lsum += s[x];
-      }
-      l_run = fmaf(l_run, alpha, lsum);
-      m_run = m_new;
+      const bool plain = full_tile && bad == 0;
 
-      // ---- keys past the context in a loaded page may hold stale data:
-      //      zero their V rows so that P = 0 cannot meet NaN in the MMA -----
-      {
-        const int z0 = max(ctx, key0);
-        const int z1 = min(((n_keys + kPS - 1) / kPS) * kPS, key0 + kBN);
-        const int nz = (z1 - z0) * (kRowBytes / 16);
-        for (int t = threadIdx.x - 64; t < nz; t += 128) {
-          const int row = z0 - key0 + t / (kRowBytes / 16);
-          const int ch = t % (kRowBytes / 16);
-          *reinterpret_cast<uint4*>(&sm.v[st][row * kRowBytes + ch * 16]) =
-              make_uint4(0, 0, 0, 0);
+      // ---- pass 1: row maximum of the raw scores ------------------------------
+      float mx = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float s[64];
+        tmem_ld64(s_addr + h * 64, s);
+        if (plain) {
+#pragma unroll
+          for (int x = 0; x < 64; x += 2) mx = fmax3(mx, s[x], s[x + 1]);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 64; ++x) {
+            const int key = key0 + h * 64 + x;
+            const bool vis =
+                key <= limit && !((bad >> ((h * 64 + x) / kPS)) & 1u);
+            mx = fmaxf(mx, vis ? s[x] : -INFINITY);
+          }
         }
       }
+      const float m_tile = mx * c;   // scale > 0, so max commutes with it
 
-      // ---- P_hi, P_lo (bf16) into the swizzled K-major layout -------------------
-      {
-        uint8_t* phi = sm.p[b][0][0] + r * kRowBytes;
-        uint8_t* plo = sm.p[b][1][0] + r * kRowBytes;
+      // ---- P.V of the previous tile must be done before P is overwritten -------
+      if (j >= 1 &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(smem_u32(&sm.o_full[t]), (j - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+
+      // ---- lazy rescale: move the running max only when it grows > 2^8 ----------
+      const bool grow = m_tile > m_run + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_new = grow ? m_tile : m_run;
+        const float alpha = fast_exp2(m_run - m_new);   // 0 when m_run = -inf
+        l_run *= alpha;
+        m_run = m_new;
+        if (j >= 1) {   // O holds the earlier tiles: rescale it in place
+          float o[64];
+          tmem_ld64(o_addr, o);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+          for (int d = 0; d < 64; ++d) o[d] *= alpha;
+          tmem_st64(o_addr, o);
+        }
+      }
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+
+      // ---- pass 2: exponentials, row sum, P_hi / P_lo into shared memory --------
+      float lsum = 0.f;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int x = half * 64 + ch * 8;
-            uint32_t hi[4], lo[4];
+      for (int h = 0; h < 2; ++h) {
+        float s[64];
+        tmem_ld64(s_addr + h * 64, s);
+        if (plain) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hi[e] = pack_bf16x2(s[x + 2 * e], s[x + 2 * e + 1]);
-              lo[e] = pack_bf16x2(s[x + 2 * e] - bf16_lo(hi[e]),
-                                  s[x + 2 * e + 1] - bf16_hi(hi[e]));
-            }
-            const int off = half * (kBM * kRowBytes) + ((ch ^ (r & 7)) * 16);
-            *reinterpret_cast<uint4*>(phi + off) =
-                make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(plo + off) =
-                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          for (int x = 0; x < 64; ++x) s[x] = fast_exp2(fmaf(s[x], c, -m_use));
+        } else {
+#pragma unroll
+          for (int x = 0; x < 64; ++x) {
+            const int key = key0 + h * 64 + x;
+            const bool vis =
+                key <= limit && !((bad >> ((h * 64 + x) / kPS)) & 1u);
+            s[x] = vis ? fast_exp2(fmaf(s[x], c, -m_use)) : 0.f;
           }
+        }
+        uint8_t* phi = sm.p[t][0][h] + r * kRowBytes;
+        uint8_t* plo = sm.p[t][1][h] + r * kRowBytes;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = s[ch * 8 + 2 * e], x1 = s[ch * 8 + 2 * e + 1];
+            lsum += x0 + x1;
+            hi[e] = pack_bf16x2(x0, x1);
+            lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+          }
+          const int off = (ch ^ (r & 7)) * 16;
+          *reinterpret_cast<uint4*>(phi + off) =
+              make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(plo + off) =
+              make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+      l_run += lsum;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[t]));
+
+      // ---- keys past the context in a loaded page may hold stale data: zero
+      //      their V rows (once per key tile, by the query tile whose P.V on
+      //      it is issued first) so that P = 0 cannot meet NaN in the MMA ----
+      if (t == 0 || j >= n_tiles_of[0]) {
+        const int z0 = max(ctx, key0);
+        const int z1 = min(n_pages * kPS, key0 + kBN);
+        const int nz = (z1 - z0) * (kRowBytes / 16);
+        for (int i = threadIdx.x - 128 * (t + 1); i < nz; i += 128) {
+          const int row = z0 - key0 + i / (kRowBytes / 16);
+          const int chn = i % (kRowBytes / 16);
+          *reinterpret_cast<uint4*>(&sm.v[st][row * kRowBytes + chn * 16]) =
+              make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b]));
-
-      // ---- fold the previous tile's P.V ------------------------------------------
-      if (j >= 1 && !fold_o(j - 1, alpha_prev)) {
-        ok = false;
-        break;
-      }
-      alpha_prev = alpha;
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[t]));
     }
-    if (ok && !fold_o(n_tiles - 1, alpha_prev)) ok = false;
-    if (!ok) {
-      if (lane == 0) flag_error(a.err, DEVERR_TIMEOUT);
+
+    // ---- wait for the last P.V, normalise and store --------------------------------
+    float o[64];
+    if (ok && my_tiles > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_full[t]),
+                                          (my_tiles - 1) & 1))) {
+      tc_fence_after();
+      tmem_ld64(o_addr, o);
+    } else {
+      if (my_tiles > 0 && lane == 0) flag_error(a.err, DEVERR_TIMEOUT);
 #pragma unroll
-      for (int d = 0; d < kD; ++d) o[d] = 0.f;
+      for (int d = 0; d < 64; ++d) o[d] = 0.f;
       l_run = 0.f;
     }
-
-    // ---- normalise and store ---------------------------------------------------
-    if (row_real) {
+    if (row_real && my_tiles > 0) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       __nv_bfloat16* dst =
-          a.out + ((size_t)(qs + q0 + qi) * a.num_q_heads + kvh * kG + hh) * kD;
+          a.out + ((size_t)(qs + qt0 + qi) * a.num_q_heads + kvh * kG + hh) * kD;
 #pragma unroll
       for (int ch = 0; ch < kD / 8; ++ch) {
         uint4 w;
@@ -408,8 +439,9 @@ cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,
   cudaError_t e = cudaFuncSetAttribute(
       paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int tiles = (a.max_query_len + kQRows - 1) / kQRows;
-  dim3 grid(a.num_kv_heads, tiles, a.num_seqs);
+  const int blocks = (a.max_query_len + kQRows * kQTiles - 1) /
+                     (kQRows * kQTiles);
+  dim3 grid(a.num_kv_heads, blocks, a.num_seqs);
   paged_prefill_kernel<<<grid, kThreads, smem, stream>>>(a, tq, tk, tv);
   return cudaGetLastError();
 }
