@@ -63,7 +63,9 @@ typedef enum {
   TV_OK = 0,
   TV_ERR_INVALID_ARG = 1,
   TV_ERR_UNSUPPORTED = 2,
-  TV_ERR_CUDA = 3
+  TV_ERR_CUDA = 3,
+  TV_ERR_SCRATCH_LIMIT = 4  /* call needs more than the library's fixed
+                               scratch (tv_paged_decode_split_static) */
 } tv_status;
 
 enum {
@@ -189,6 +191,40 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
                            int num_kv_heads, int head_dim, int page_size,
                            int64_t num_pages, float scale, uint32_t* err,
                            void* stream);
+
+/*
+ * tv_paged_decode_split_static -- tv_paged_decode_split followed by
+ * tv_split_merge in one call that allocates nothing: the fp32 partials go to
+ * a fixed array inside the library instead of caller buffers.  The source
+ * pages have no counterpart of this call; it exists for callers that cannot
+ * allocate on the decode path: engines that give (almost) all device memory
+ * to the KV page pool at start-up and allow no allocation while serving,
+ * step loops that cannot afford cudaMalloc/cudaFree (which may block and
+ * synchronise the device), and plain C hosts with no device allocator.
+ *   out and every other argument: as tv_paged_decode_split / tv_split_merge;
+ *   out [num_seqs][num_q_heads][head_dim] bf16 receives the merged result.
+ * Limits and sharing:
+ *   - the array holds TV_STATIC_SCRATCH_FLOATS floats (32 MiB) per device
+ *     and stays allocated on every GPU that loads the library until exit;
+ *   - a call needs num_seqs * num_q_heads * max_partitions * (head_dim + 1)
+ *     floats; a larger one returns TV_ERR_SCRATCH_LIMIT before any launch;
+ *   - every call on a device shares the array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero: each call rewrites
+ *     every partial it reads); calls that overlap on the GPU (unordered
+ *     streams) race on it;
+ *   - the first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ * Returns TV_ERR_CUDA when that lookup fails.
+ */
+#define TV_STATIC_SCRATCH_FLOATS (1 << 23)
+
+tv_status tv_paged_decode_split_static(
+    void* out, const void* q, const void* k_pool, const void* v_pool,
+    const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int page_size, int64_t num_pages,
+    float scale, int partition_tokens, int max_partitions, uint32_t* err,
+    void* stream);
 
 #ifdef __cplusplus
 }

@@ -18,7 +18,9 @@ LIB_PATH = os.path.join(_PKG, "libtv.so")
 
 TV_OK = 0
 STATUS = {0: "TV_OK", 1: "TV_ERR_INVALID_ARG", 2: "TV_ERR_UNSUPPORTED",
-          3: "TV_ERR_CUDA"}
+          3: "TV_ERR_CUDA", 4: "TV_ERR_SCRATCH_LIMIT"}
+TV_ERR_SCRATCH_LIMIT = 4
+STATIC_SCRATCH_FLOATS = 1 << 23   # TV_STATIC_SCRATCH_FLOATS in include/tv.h
 DEVERR_BAD_SLOT = 1 << 0
 DEVERR_BAD_PAGE = 1 << 1
 DEVERR_BAD_CONTEXT = 1 << 2
@@ -40,6 +42,9 @@ SIGNATURES = {
     "tv_split_merge": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "tv_paged_prefill": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _I, _I,
                               _I, _I, _I, _I, _I64, _F, _P, _P]),
+    "tv_paged_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I,
+                                          _I, _I, _I, _I64, _F, _I, _I, _P,
+                                          _P]),
 }
 
 _lib = None
@@ -216,3 +221,31 @@ def tv_paged_prefill(out, q, query_start_loc, k_pool, v_pool, block_tables,
         _ptr(context_lens), b, int(max_query_len), hq, hkv, d, page_size,
         num_pages, float(scale), _ptr(err), _stream(stream)),
         "tv_paged_prefill")
+
+
+def tv_paged_decode_split_static(out, q, k_pool, v_pool, block_tables,
+                                 context_lens, scale, partition_tokens,
+                                 max_partitions, err=None, stream=None):
+    """Split-KV decode + merge into out[B][Hq][D] (bf16) without any
+    caller-side scratch: the partials live in the library's fixed device
+    array (for callers that cannot allocate on the decode path).  Raises
+    TVError with TV_ERR_SCRATCH_LIMIT when B * Hq * max_partitions * (D + 1)
+    exceeds STATIC_SCRATCH_FLOATS."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_pool", k_pool),
+                 ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != b:
+        raise ValueError("shape mismatch")
+    _check(lib.tv_paged_decode_split_static(
+        _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), b, hq, hkv, d, page_size,
+        num_pages, float(scale), int(partition_tokens), int(max_partitions),
+        _ptr(err), _stream(stream)), "tv_paged_decode_split_static")

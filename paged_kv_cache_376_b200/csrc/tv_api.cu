@@ -121,6 +121,7 @@ const char* tv_status_string(tv_status status) {
     case TV_ERR_INVALID_ARG: return "TV_ERR_INVALID_ARG";
     case TV_ERR_UNSUPPORTED: return "TV_ERR_UNSUPPORTED";
     case TV_ERR_CUDA: return "TV_ERR_CUDA";
+    case TV_ERR_SCRATCH_LIMIT: return "TV_ERR_SCRATCH_LIMIT";
   }
   return "TV_ERR_UNKNOWN";
 }
