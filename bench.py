@@ -5,8 +5,10 @@
                     [--workload llama|mix|long|prefill|tiny]
 
 A step is one pass of the hot path over one batch:
-  llama / mix / tiny : tv_kv_append of one token per sequence, then
-                       tv_paged_decode over the whole paged context;
+  llama / mix / tiny : the decode step -- append one token per sequence and
+                       attend over the whole paged context -- as the single
+                       fused launch tv_paged_decode_append (--unfused: the
+                       two calls tv_kv_append + tv_paged_decode);
   long               : tv_kv_append, tv_paged_decode_split (512-token
                        partitions), tv_split_merge;
   prefill            : tv_kv_append of the 512-token chunks, then
@@ -54,6 +56,25 @@ def _peaks():
                 "fallback")
 
 
+def _traffic(kernel, workload_name):
+    """DRAM bytes per launch of `kernel` on this workload from the committed
+    ncu capture (profiles/traffic.json), or None when there is none or when a
+    source file of the kernel has changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(f"{kernel}@{workload_name}")
+        if not entry:
+            return None
+        for path, digest in entry["sources"].items():
+            with open(os.path.join(ROOT, path), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        return int(entry["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def _workload(name):
     from paged_kv_cache_376_b200 import workloads as W
     return {"llama": W.llama_decode, "mix": W.continuous_mix,
@@ -61,14 +82,15 @@ def _workload(name):
             "tiny": W.tiny_decode}[name]()
 
 
-def _config(wl, name):
+def _config(wl, name, unfused=False):
     cfg = {"workload": wl.name, "batch": wl.num_seqs,
            "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
            "head_dim": wl.head_dim, "page_size": wl.page_size,
            "num_pages": wl.num_pages,
            "context_tokens": int(wl.context_lens.sum())}
     if name in ("llama", "mix", "tiny"):
-        cfg["step"] = "tv_kv_append + tv_paged_decode"
+        cfg["step"] = ("tv_kv_append + tv_paged_decode" if unfused else
+                       "tv_paged_decode_append (fused append + decode)")
     elif name == "long":
         cfg["step"] = ("tv_kv_append + tv_paged_decode_split + "
                        "tv_split_merge")
@@ -144,7 +166,7 @@ class TVRunner:
     """Device buffers and the calls of one step, marshalled once so that the
     host submits a step in a few microseconds."""
 
-    def __init__(self, wl, name, device):
+    def __init__(self, wl, name, device, unfused=False):
         import torch
         from paged_kv_cache_376_b200 import _lib
         from paged_kv_cache_376_b200.device import upload
@@ -154,7 +176,8 @@ class TVRunner:
         self.db = db = upload(wl, device)
         self.out = torch.empty_like(db.q)
         self.kind = ("prefill" if name == "prefill" else
-                     "split" if name == "long" else "decode")
+                     "split" if name == "long" else
+                     "decode" if unfused else "fused")
         if self.kind == "split":
             maxp = wl.max_partitions()
             b, hq, d = db.q.shape
@@ -176,6 +199,20 @@ class TVRunner:
         lib, db, wl = self.lib, self.db, self.wl
         s = self.stream.cuda_stream
         num_pages, ps, hkv, d = db.k_pool.shape
+        b, hq = db.context_lens.shape[0], db.q.shape[1]
+        mb = db.block_tables.shape[1]
+        if self.kind == "fused":
+            if timing is not None:
+                timing[0].record(self.stream)
+            st = lib.tv_paged_decode_append(
+                self._p(self.out), self._p(db.q), self._p(db.k_new),
+                self._p(db.v_new), self._p(db.k_pool), self._p(db.v_pool),
+                self._p(db.block_tables), mb, self._p(db.context_lens), b, hq,
+                hkv, d, ps, num_pages, wl.scale, self._p(db.err), s)
+            assert st == 0, st
+            if timing is not None:
+                timing[1].record(self.stream)
+            return
         st = lib.tv_kv_append(
             self._p(db.k_new), self._p(db.v_new), self._p(db.slot_mapping),
             db.k_new.shape[0], self._p(db.k_pool), self._p(db.v_pool),
@@ -183,8 +220,6 @@ class TVRunner:
         assert st == 0, st
         if timing is not None:
             timing[0].record(self.stream)
-        b, hq = db.context_lens.shape[0], db.q.shape[1]
-        mb = db.block_tables.shape[1]
         if self.kind == "decode":
             st = lib.tv_paged_decode(
                 self._p(self.out), self._p(db.q), self._p(db.k_pool),
@@ -216,15 +251,21 @@ class TVRunner:
             assert st == 0, st
 
     def launches_per_step(self):
-        return 3 if self.kind == "split" else 2
+        return {"split": 3, "fused": 1}.get(self.kind, 2)
 
     # -- end to end: host inputs in, host result out, through the C ABI ------
     def setup_e2e(self):
         torch = self.torch
         db = self.db
         self.h_in = {}
-        for name in ("q", "k_new", "v_new", "slot_mapping", "block_tables",
-                     "context_lens", "query_start_loc"):
+        names = {"fused": ("q", "k_new", "v_new", "block_tables",
+                           "context_lens"),
+                 "prefill": ("q", "k_new", "v_new", "slot_mapping",
+                             "block_tables", "context_lens",
+                             "query_start_loc")}.get(
+            self.kind, ("q", "k_new", "v_new", "slot_mapping",
+                        "block_tables", "context_lens"))
+        for name in names:
             t = getattr(db, name)
             self.h_in[name] = torch.empty(t.shape, dtype=t.dtype,
                                           pin_memory=True).copy_(t.cpu())
@@ -257,7 +298,7 @@ def run_tv(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     wl = _workload(args.workload)
-    runner = TVRunner(wl, args.workload, device)
+    runner = TVRunner(wl, args.workload, device, unfused=args.unfused)
     per_step, unit, seqs = _units(wl, args.workload)
     hbm, tfl, tfl_sus, peak_src = _peaks()
     K, Wm = args.steps, args.warmup
@@ -311,9 +352,12 @@ def run_tv(args, rank, world, local_rank):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, device)
     h2d, d2h = runner.e2e_bytes()
 
-    value = world * per_step * K / (ms_max / 1e3)
+    value = whole_job_rate(per_step, K, ms_max, world)
     step_ms = ms_max / K
     kern_per_launch = per_step / (kern_ms_max / 1e3)     # GB/s or TFLOP/s
+    kernel_name = {"decode": "tv_paged_decode", "split":
+                   "tv_paged_decode_split", "prefill": "tv_paged_prefill",
+                   "fused": "tv_paged_decode_append"}[runner.kind]
     if unit == "GB/s":
         peak, bound, src = hbm, "hbm", peak_src
     else:
@@ -326,10 +370,10 @@ def run_tv(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, shuffled "
         "page pool)",
-        "config": dict(_config(wl, args.workload),
+        "config": dict(_config(wl, args.workload, args.unfused),
                        parallelism=f"replicas{world}" if world > 1
                        else "single GPU"),
-        "seq_steps_per_s": round(world * seqs * K / (ms_max / 1e3), 1),
+        "seq_steps_per_s": round(whole_job_rate(seqs, K, ms_max, world), 1),
         "hbm_frac" if unit == "GB/s" else "tensor_frac":
             round(value / world / peak, 4),
         "roofline": {
@@ -337,13 +381,12 @@ def run_tv(args, rank, world, local_rank):
             "peak": peak, "unit": unit, "frac": round(kern_per_launch / peak,
                                                       4),
             "peak_source": f"{src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
-            "kernel": {"decode": "tv_paged_decode", "split":
-                       "tv_paged_decode_split", "prefill":
-                       "tv_paged_prefill"}[runner.kind],
+            "kernel": kernel_name,
             "kernel_ms": round(kern_ms_max, 6),
-            "traffic": None,
+            "traffic": _traffic(kernel_name, wl.name),
+            "traffic_unit": "bytes per launch (ncu dram read + write)",
         },
-        "e2e": {"value": round(world * per_step * K / (e2e_ms / 1e3), 3),
+        "e2e": {"value": round(whole_job_rate(per_step, K, e2e_ms, world), 3),
                 "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": K * runner.launches_per_step(),
@@ -366,6 +409,9 @@ def _gpu_index(local_rank):
 
 
 def _max_over_ranks(x, world, device):
+    """The slowest rank's time: every rank calls this with its own device
+    time; the result is the same on all ranks (a host-side timing reduction,
+    not part of the data path)."""
     if world == 1:
         return x
     import torch
@@ -373,6 +419,12 @@ def _max_over_ranks(x, world, device):
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank, steps, ms_max, world):
+    """Whole-job throughput: every rank runs its own replica of the batch,
+    so the job processes world x units per step; time is the slowest rank's."""
+    return world * units_per_step_per_rank * steps / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------ oracle arm --
@@ -502,6 +554,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama",
                     choices=["llama", "mix", "long", "prefill", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="decode step as tv_kv_append + tv_paged_decode")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

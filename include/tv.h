@@ -127,6 +127,31 @@ tv_status tv_paged_decode(void* out, const void* q, const void* k_pool,
                           float scale, uint32_t* err, void* stream);
 
 /*
+ * tv_paged_decode_append -- the whole decode step in one launch: append the
+ * new token of every sequence at position context_lens[s]-1 (its slot found
+ * through the block table) and attend over the cache, i.e. the result of
+ * tv_kv_append with slot = block_tables[s][(ctx-1)/16]*16 + (ctx-1)%16
+ * followed by tv_paged_decode ([P1] "推理流程": compute the new token's K,V,
+ * append them to the cache, then attend).  The new row is written to the
+ * pools and used directly from shared memory, never read back from HBM.
+ *   k_new, v_new   [num_seqs][num_kv_heads][head_dim] bf16
+ *   k_pool, v_pool updated in place (one row per sequence and KV head)
+ *   other arguments as tv_paged_decode; context_lens[s] >= 1 counts the new
+ *   token.  A sequence with context 0 appends nothing and outputs zeros.
+ * The appended slot must not be read by another sequence of the same call
+ * (a shared prefix page is never the page a token is appended to).
+ */
+tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
+                                 const void* v_new, void* k_pool, void* v_pool,
+                                 const int32_t* block_tables,
+                                 int max_blocks_per_seq,
+                                 const int32_t* context_lens, int num_seqs,
+                                 int num_q_heads, int num_kv_heads,
+                                 int head_dim, int page_size,
+                                 int64_t num_pages, float scale,
+                                 uint32_t* err, void* stream);
+
+/*
  * tv_paged_decode_split -- tv_paged_decode restricted to logical key
  * partitions p = [p*partition_tokens, (p+1)*partition_tokens) of each
  * context (the blockwise online softmax of [P1] "在线Softmax"):

@@ -37,6 +37,8 @@ SIGNATURES = {
                           _P]),
     "tv_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                              _I64, _F, _P, _P]),
+    "tv_paged_decode_append": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
+                                    _I, _I, _I, _I, _I64, _F, _P, _P]),
     "tv_paged_decode_split": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I,
                                    _I, _I, _I, _I64, _F, _I, _I, _P, _P]),
     "tv_split_merge": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -148,6 +150,33 @@ def tv_paged_decode(out, q, k_pool, v_pool, block_tables, context_lens,
         block_tables.shape[1], _ptr(context_lens), b, hq, hkv, d, page_size,
         num_pages, float(scale), _ptr(err), _stream(stream)),
         "tv_paged_decode")
+
+
+def tv_paged_decode_append(out, q, k_new, v_new, k_pool, v_pool,
+                           block_tables, context_lens, scale, err=None,
+                           stream=None):
+    """Fused decode step: append k_new/v_new [B][Hkv][D] at position
+    context_len-1 of each sequence (slot from the block table) and write the
+    attention of q[B][Hq][D] over the cache into out[B][Hq][D]."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_new", k_new), ("v_new", v_new),
+                 ("k_pool", k_pool), ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != b or \
+            k_new.shape != (b, hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch")
+    _check(lib.tv_paged_decode_append(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+        _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), b, hq, hkv, d, page_size, num_pages, float(scale),
+        _ptr(err), _stream(stream)), "tv_paged_decode_append")
 
 
 def tv_paged_decode_split(partial_out, partial_lse, q, k_pool, v_pool,

@@ -26,6 +26,11 @@
 //  * The split variant writes the normalised partial output and the natural
 //    log-sum-exp of each 512-token (or any multiple of 16) partition; the
 //    merge kernel (split_merge.cu) combines them.
+//  * The append variant fuses the KV append of the decode step ("推理流程":
+//    compute the new token's K,V, append them, then attend): the warp that
+//    owns the page holding position context_len-1 writes the new token's row
+//    of its KV head into the pool and into its staged copy of that page, so
+//    the step is one launch and the new row is never read back from HBM.
 #include "tv_device.cuh"
 #include "tv_kernels.h"
 
@@ -53,7 +58,7 @@ struct Combine {  // per-warp results handed to the final combine
   float acc[kWarps][G][kD];
 };
 
-template <int G, int kStages, bool kSplit>
+template <int G, int kStages, bool kSplit, bool kAppend>
 __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     paged_decode_kernel(const DecodeArgs a,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -92,6 +97,24 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int my_n = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
   const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq +
                       first_page + warp;
+
+  // ---- fused append: the new token is at position ctx-1 (unsplit kernel) ---
+  int app_i = -1;            // local page index of the appended row, this warp
+  int app_r = 0;             // its row within the page
+  uint4 app_row = make_uint4(0, 0, 0, 0);  // lanes 0-7: K chunk, 8-15: V chunk
+  if (kAppend && ctx > 0) {
+    const int lp = (ctx - 1) / kPS;
+    if (lp % kWarps == warp) {
+      app_i = lp / kWarps;
+      app_r = (ctx - 1) % kPS;
+      if (lane < 16) {
+        const __nv_bfloat16* src =
+            (lane < 8 ? a.k_new : a.v_new) +
+            ((size_t)seq * gridDim.x + kvh) * kD + chk * 8;
+        app_row = *reinterpret_cast<const uint4*>(src);
+      }
+    }
+  }
 
   // ---- barriers ------------------------------------------------------------
   if (lane == 0) {
@@ -180,6 +203,19 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     }
     const uint8_t* kbase = &sm.ring[warp][stage][0];
     const uint8_t* vbase = kbase + kSliceBytes;
+    if (kAppend && i == app_i) {
+      // the staged page now gets the new row; the pool keeps it for later
+      if (page_ok && lane < 16) {
+        uint8_t* dst = &sm.ring[warp][stage][(lane < 8 ? 0 : kSliceBytes) +
+                                             app_r * kRowBytes + chk * 16];
+        *reinterpret_cast<uint4*>(dst) = app_row;
+        __nv_bfloat16* pool = lane < 8 ? a.k_pool_w : a.v_pool_w;
+        *reinterpret_cast<uint4*>(
+            pool + (((size_t)pid * kPS + app_r) * gridDim.x + kvh) * kD +
+            chk * 8) = app_row;
+      }
+      __syncwarp();
+    }
 
     // ---- scores: token it*4+grp, head my_head ---------------------------------
     float s[4];
@@ -357,11 +393,11 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   }
 }
 
-template <int G, int kStages, bool kSplit>
+template <int G, int kStages, bool kSplit, bool kAppend>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk,
                      const CUtensorMap& tv, int num_kv_heads, int num_seqs,
                      int parts, cudaStream_t stream) {
-  auto kern = paged_decode_kernel<G, kStages, kSplit>;
+  auto kern = paged_decode_kernel<G, kStages, kSplit, kAppend>;
   const int smem = sizeof(DecodeSmem<kStages>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -378,13 +414,17 @@ cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
                                 int num_seqs, int group, bool split,
                                 int parts, cudaStream_t stream) {
   constexpr int S = 3;
+  const bool append = a.k_new != nullptr;
   switch (group) {
-#define TV_CASE(G)                                                         \
-  case G:                                                                  \
-    return split ? launch_g<G, S, true>(a, tk, tv, num_kv_heads, num_seqs, \
-                                        parts, stream)                     \
-                 : launch_g<G, S, false>(a, tk, tv, num_kv_heads,          \
-                                         num_seqs, 1, stream);
+#define TV_CASE(G)                                                          \
+  case G:                                                                   \
+    if (split)                                                              \
+      return launch_g<G, S, true, false>(a, tk, tv, num_kv_heads, num_seqs, \
+                                         parts, stream);                    \
+    return append ? launch_g<G, S, false, true>(a, tk, tv, num_kv_heads,    \
+                                                num_seqs, 1, stream)        \
+                  : launch_g<G, S, false, false>(a, tk, tv, num_kv_heads,   \
+                                                 num_seqs, 1, stream);
     TV_CASE(1)
     TV_CASE(2)
     TV_CASE(4)

@@ -153,6 +153,7 @@ tv_status tv_kv_append(const void* k_new, const void* v_new,
 
 static tv_status decode_common(void* out, float* partial_out,
                                float* partial_lse, const void* q,
+                               const void* k_new, const void* v_new,
                                const void* k_pool, const void* v_pool,
                                const int32_t* block_tables,
                                int max_blocks_per_seq,
@@ -181,6 +182,10 @@ static tv_status decode_common(void* out, float* partial_out,
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
       (!split && !aligned16(out)))
     return TV_ERR_INVALID_ARG;
+  if ((k_new != nullptr) != (v_new != nullptr) || (split && k_new))
+    return TV_ERR_INVALID_ARG;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    return TV_ERR_INVALID_ARG;
 
   CUtensorMap tk, tvm;
   st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
@@ -195,6 +200,10 @@ static tv_status decode_common(void* out, float* partial_out,
   a.partial_out = partial_out;
   a.partial_lse = partial_lse;
   a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.k_pool_w = static_cast<__nv_bfloat16*>(const_cast<void*>(k_pool));
+  a.v_pool_w = static_cast<__nv_bfloat16*>(const_cast<void*>(v_pool));
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.err = err;
@@ -215,10 +224,26 @@ tv_status tv_paged_decode(void* out, const void* q, const void* k_pool,
                           int num_seqs, int num_q_heads, int num_kv_heads,
                           int head_dim, int page_size, int64_t num_pages,
                           float scale, uint32_t* err, void* stream) {
-  return decode_common(out, nullptr, nullptr, q, k_pool, v_pool, block_tables,
-                       max_blocks_per_seq, context_lens, num_seqs,
-                       num_q_heads, num_kv_heads, head_dim, page_size,
-                       num_pages, scale, 0, 1, false, err, stream);
+  return decode_common(out, nullptr, nullptr, q, nullptr, nullptr, k_pool,
+                       v_pool, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, 0, 1, false, err, stream);
+}
+
+tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
+                                 const void* v_new, void* k_pool, void* v_pool,
+                                 const int32_t* block_tables,
+                                 int max_blocks_per_seq,
+                                 const int32_t* context_lens, int num_seqs,
+                                 int num_q_heads, int num_kv_heads,
+                                 int head_dim, int page_size,
+                                 int64_t num_pages, float scale,
+                                 uint32_t* err, void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return TV_ERR_INVALID_ARG;
+  return decode_common(out, nullptr, nullptr, q, k_new, v_new, k_pool, v_pool,
+                       block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, 0, 1, false, err, stream);
 }
 
 tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
@@ -232,8 +257,8 @@ tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
                                 int64_t num_pages, float scale,
                                 int partition_tokens, int max_partitions,
                                 uint32_t* err, void* stream) {
-  return decode_common(nullptr, partial_out, partial_lse, q, k_pool, v_pool,
-                       block_tables, max_blocks_per_seq, context_lens,
+  return decode_common(nullptr, partial_out, partial_lse, q, nullptr, nullptr,
+                       k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
                        num_seqs, num_q_heads, num_kv_heads, head_dim,
                        page_size, num_pages, scale, partition_tokens,
                        max_partitions, true, err, stream);

@@ -13,6 +13,10 @@ struct DecodeArgs {
   float* partial_out;            // [B][Hq][maxP][D]      (split)
   float* partial_lse;            // [B][Hq][maxP]         (split)
   const __nv_bfloat16* q;        // [B][Hq][D]
+  const __nv_bfloat16* k_new;    // [B][Hkv][D] (fused append; else null)
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool_w;       // pools, written by the fused append
+  __nv_bfloat16* v_pool_w;
   const int32_t* block_tables;   // [B][max_blocks_per_seq]
   const int32_t* context_lens;   // [B]
   uint32_t* err;                 // nullable

@@ -140,3 +140,55 @@ def test_context_beyond_block_table_is_clamped_and_flagged():
     db.context_lens[0] = 10_000
     gpu_decode(db, wl.scale)
     assert err_word(db) & _lib.DEVERR_BAD_CONTEXT
+
+
+# ---- fused append + decode (one launch per decode step) ---------------------
+
+def _fused(wl):
+    db = upload(wl)
+    out = torch.empty_like(db.q)
+    _lib.tv_paged_decode_append(out, db.q, db.k_new, db.v_new, db.k_pool,
+                                db.v_pool, db.block_tables, db.context_lens,
+                                wl.scale, err=db.err)
+    torch.cuda.synchronize()
+    return db, out
+
+
+@pytest.mark.parametrize("make", [W.tiny_decode, W.llama_decode,
+                                  W.continuous_mix],
+                         ids=["tiny", "llama", "mix"])
+def test_fused_append_decode_matches_oracle_and_appends(make):
+    wl = make()
+    db, out = _fused(wl)
+    kp, vp = oracle_after_append(wl)
+    # the pools hold exactly what a separate append would have written
+    np.testing.assert_array_equal(bf16_bits(db.k_pool), kp)
+    np.testing.assert_array_equal(bf16_bits(db.v_pool), vp)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, f"fused {wl.name}")
+    assert err_word(db) == 0
+
+
+def test_fused_equals_append_then_decode_bitwise():
+    lens = [1, 2, 16, 17, 31, 32, 33, 100, 1000, 2049]
+    wl = W.decode_workload(lens, seed=55)
+    _, fused = _fused(wl)
+    db = upload(wl)
+    gpu_append(db)
+    sep = gpu_decode(db, wl.scale)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bf16_bits(fused), bf16_bits(sep))
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 4)],
+                         ids=["mha", "gqa2", "gqa8"])
+def test_fused_group_sizes(hq, hkv):
+    lens = [1, 15, 16, 17, 300]
+    wl = W.decode_workload(lens, seed=56, num_q_heads=hq, num_kv_heads=hkv)
+    db, out = _fused(wl)
+    kp, vp = oracle_after_append(wl)
+    np.testing.assert_array_equal(bf16_bits(db.k_pool), kp)
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, f"fused hq={hq} hkv={hkv}")
