@@ -166,7 +166,7 @@ class TVRunner:
     """Device buffers and the calls of one step, marshalled once so that the
     host submits a step in a few microseconds."""
 
-    def __init__(self, wl, name, device, unfused=False):
+    def __init__(self, wl, name, device, unfused=False, split_tokens=0):
         import torch
         from paged_kv_cache_376_b200 import _lib
         from paged_kv_cache_376_b200.device import upload
@@ -176,9 +176,11 @@ class TVRunner:
         self.db = db = upload(wl, device)
         self.out = torch.empty_like(db.q)
         self.kind = ("prefill" if name == "prefill" else
-                     "split" if name == "long" else
+                     "split" if name == "long" or split_tokens else
                      "decode" if unfused else "fused")
         if self.kind == "split":
+            if split_tokens:
+                wl.partition_tokens = split_tokens
             maxp = wl.max_partitions()
             b, hq, d = db.q.shape
             self.po = torch.empty((b, hq, maxp, d), dtype=torch.float32,
@@ -298,7 +300,8 @@ def run_tv(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     wl = _workload(args.workload)
-    runner = TVRunner(wl, args.workload, device, unfused=args.unfused)
+    runner = TVRunner(wl, args.workload, device, unfused=args.unfused,
+                      split_tokens=args.split_tokens)
     per_step, unit, seqs = _units(wl, args.workload)
     hbm, tfl, tfl_sus, peak_src = _peaks()
     K, Wm = args.steps, args.warmup
@@ -556,6 +559,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="decode step as tv_kv_append + tv_paged_decode")
+    ap.add_argument("--split-tokens", type=int, default=0,
+                    help="decode step as tv_kv_append + tv_paged_decode_split "
+                         "(partitions of this many tokens) + tv_split_merge")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -17,24 +17,31 @@
 //    K/V tile, and the tensor core alternates between them while the other
 //    tile's softmax runs.  q arrives by one 3-D TMA box {64 d, 4 heads, 32
 //    rows} per tile.
-//  * Keys come in tiles of 128 = 8 pages; each page of one KV head (16 rows x
-//    128 B) is one 2-D TMA box, 128-byte swizzled, so 8 boxes at 2 KB
+//  * Keys come in tiles of 64 = 4 pages; each page of one KV head (16 rows x
+//    128 B) is one 2-D TMA box, 128-byte swizzled, so 4 boxes at 2 KB
 //    offsets form exactly the canonical K-major SW128 operand.  Pages past
 //    the range (or with a bad id) are read at an out-of-range coordinate and
 //    arrive as zeros.
-//  * warp 0: TMA producer (q once, K/V through a 2-stage ring).
+//  * P never goes through shared memory: the softmax writes P (bf16) back
+//    into the tensor-memory columns its S came from, and P.V is issued with
+//    A read from tensor memory, so the tensor core's shared-memory reads are
+//    only q, K and V (with P in shared memory the MMAs were starved on
+//    shared-memory bandwidth).  S/P is double-buffered per query tile and
+//    K/V run through an 8-stage ring, so the MMA thread issues S_{j+1} while
+//    tile j is exponentiated and P_j.V_j while tile j+1 is.
+//  * warp 0: TMA producer (q once, K/V ring).
 //    warp 1: tensor-memory allocation and the single MMA-issuing thread:
-//      S_t = Q_t K_j^T (M128 N128 K16 x4) into tile t's S columns, then
-//      O_t += P_t V_j (M128 N64 K16 x8, once for P_hi and once for P_lo;
-//      V read as an MN-major operand) accumulated in tile t's O columns.
+//      S_t = Q_t K_j^T (M128 N64 K16 x4) into one of tile t's two S/P
+//      buffers, then O_t += P_t V_j (M128 N64 K16 x4, once for P_hi and once
+//      for P_lo; V read as an MN-major operand) accumulated in tile t's O.
 //    warps 4-7 / 8-11: softmax of tile A / B.  Thread = one MMA row = one
-//      (query, head).  Pass 1 reads its 128 scores from tensor memory and
-//      takes their maximum; the running maximum moves only when it grows by
-//      more than 2^8 (then O and l are rescaled in place, which is rare), so
-//      O stays in tensor memory across key tiles.  Pass 2 re-reads the
-//      scores, exponentiates, sums, and writes P into the swizzled K-major
-//      layout the MMA reads.  The causal mask is applied only to the tiles
-//      that cross the diagonal.
+//      (query, head).  It reads its 64 scores from tensor memory in one load,
+//      takes their maximum, moves the running maximum only when it grows by
+//      more than 2^8 (then O and l are rescaled in place, which is rare, so O
+//      stays in tensor memory across key tiles), exponentiates, sums, and
+//      stores P_hi / P_lo into the same 64 columns (32 each, two bf16 per
+//      column).  The causal mask is applied only to the tiles that cross the
+//      diagonal.
 //  * P is split as P_hi = bf16(p), P_lo = bf16(p - P_hi) so the PV product
 //    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
 //    operands); a single bf16 P carries 8 bits, which is not enough for rows
@@ -52,17 +59,16 @@ constexpr int kG = 4;                    // query heads per KV head
 constexpr int kQRows = 32;               // query rows per MMA tile
 constexpr int kQTiles = 2;               // MMA tiles per CTA (A, B)
 constexpr int kBM = kQRows * kG;         // 128 MMA rows
-constexpr int kBN = 128;                 // keys per tile
-constexpr int kPagesPerTile = kBN / kPS; // 8
-constexpr int kST = 2;                   // K/V ring depth
+constexpr int kBN = 64;                  // keys per tile
+constexpr int kPagesPerTile = kBN / kPS; // 4
+constexpr int kST = 8;                   // K/V ring depth
 constexpr int kRowBytes = kD * 2;        // 128
-constexpr int kTileBytes = kBN * kRowBytes;  // 16 KB
+constexpr int kTileBytes = kBN * kRowBytes;  // 8 KB
 constexpr int kPageBytes = kPS * kRowBytes;  // 2 KB
-constexpr int kHalfBytes = kBM * kRowBytes;  // one 64-key half of P: 16 KB
 constexpr int kThreads = 384;
 constexpr int kTmemCols = 512;
-constexpr int kSCol = 0;                 // S of tile t: columns [128t, 128t+128)
-constexpr int kOCol = kQTiles * kBN;     // O of tile t: [256 + 64t, +64)
+constexpr int kSCol = 0;   // S/P of tile t, buffer b: columns [64(2t+b), +64)
+constexpr int kOCol = kQTiles * 2 * kBN;  // O of tile t: [256 + 64t, +64)
 constexpr float kRescaleThreshold = 8.f; // log2 units: rescale when max grows > 2^8
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
@@ -70,13 +76,11 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct PrefillSmem {
   alignas(1024) uint8_t q[kQTiles][kBM * kRowBytes];        // 32 KB
-  alignas(1024) uint8_t k[kST][kTileBytes];                 // 32 KB
-  alignas(1024) uint8_t v[kST][kTileBytes];                 // 32 KB
-  // P = P_hi + P_lo, both bf16: [tile][hi/lo][key half][128 rows x 128 B]
-  alignas(1024) uint8_t p[kQTiles][2][2][kHalfBytes];       // 128 KB
+  alignas(1024) uint8_t k[kST][kTileBytes];                 // 64 KB
+  alignas(1024) uint8_t v[kST][kTileBytes];                 // 64 KB
   alignas(8) uint64_t q_full;
   uint64_t kv_full[kST], kv_empty[kST];
-  uint64_t s_full[kQTiles], s_free[kQTiles], p_full[kQTiles], o_full[kQTiles];
+  uint64_t s_full[kQTiles][2], p_full[kQTiles][2], o_done[kQTiles][2];
   uint32_t tmem_base;
   uint32_t bad_pages[kST];
 };
@@ -133,10 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
     for (int t = 0; t < kQTiles; ++t) {
-      mbar_init(smem_u32(&sm.s_full[t]), 1);
-      mbar_init(smem_u32(&sm.s_free[t]), 4);
-      mbar_init(smem_u32(&sm.p_full[t]), 4);
-      mbar_init(smem_u32(&sm.o_full[t]), 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(smem_u32(&sm.s_full[t][b]), 1);
+        mbar_init(smem_u32(&sm.p_full[t][b]), 4);
+        mbar_init(smem_u32(&sm.o_done[t][b]), 1);
+      }
     }
     fence_mbar_init();
   }
@@ -199,8 +204,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= MMA issuer =======================================
     if (lane == 0) {
       bool ok = mbar_wait(smem_u32(&sm.q_full), 0);
+      // Barrier X[t][b] serves the tiles j with j % 2 == b; its (j / 2)-th
+      // phase belongs to tile j, so a wait for tile j uses parity (j >> 1) & 1.
       auto issue_qk = [&](int t, int j) -> bool {
-        if (j >= 1 && !mbar_wait(smem_u32(&sm.s_free[t]), (j - 1) & 1))
+        const int b = j & 1;
+        // S/P buffer b holds P of tile j - 2 until its P.V has completed
+        if (j >= 2 &&
+            !mbar_wait(smem_u32(&sm.o_done[t][b]), ((j - 2) >> 1) & 1))
           return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q[t]);
@@ -209,31 +219,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kD / 16; ++k) {
           const uint64_t ad = smem_desc_sw128(q_addr + k * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_addr + k * 32, 16, 1024);
-          tc_mma_bf16(tmem + kSCol + t * kBN, ad, bd, kIdescQK, k > 0);
+          tc_mma_bf16(tmem + kSCol + (2 * t + b) * kBN, ad, bd, kIdescQK,
+                      k > 0);
         }
-        tc_commit(smem_u32(&sm.s_full[t]));
+        tc_commit(smem_u32(&sm.s_full[t][b]));
         return true;
       };
       auto issue_pv = [&](int t, int j) -> bool {
-        if (!mbar_wait(smem_u32(&sm.p_full[t]), j & 1)) return false;
+        const int b = j & 1;
+        if (!mbar_wait(smem_u32(&sm.p_full[t][b]), (j >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sm.v[j % kST]);
+        const uint32_t p_col = tmem + kSCol + (2 * t + b) * kBN;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
-          const uint32_t p_addr = smem_u32(sm.p[t][part][0]);
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k) {
-            // A = P: K-major; keys [16k, 16k+16) sit in half k/4, byte 32*(k%4)
-            const uint64_t ad = smem_desc_sw128(
-                p_addr + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 1024);
+            // A = P in tensor memory: keys [16k, 16k+16) = 8 columns
+            const uint32_t a_tmem = p_col + part * (kBN / 2) + k * 8;
             // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
             const uint64_t bd =
                 smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
-            tc_mma_bf16(tmem + kOCol + t * kD, ad, bd, kIdescPV,
-                        (j | part | k) != 0);
+            tc_mma_bf16_ts(tmem + kOCol + t * kD, a_tmem, bd, kIdescPV,
+                           (j | part | k) != 0);
           }
         }
-        tc_commit(smem_u32(&sm.o_full[t]));
+        tc_commit(smem_u32(&sm.o_done[t][b]));
         return true;
       };
       for (int j = 0; ok && j <= n_tiles; ++j) {
@@ -267,55 +278,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int limit = row_real ? P + qt0 + qi : ctx - 1;  // last visible key
     const int my_tiles = n_tiles_of[t];
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + kSCol + t * kBN;
+    const uint32_t s_addr = tmem + lane_base + kSCol + 2 * t * kBN;
     const uint32_t o_addr = tmem + lane_base + kOCol + t * kD;
     const float c = a.scale_log2;
 
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < my_tiles; ++j) {
+      const int b = j & 1;
       const int st = j % kST;
       const int key0 = j * kBN;
       // every row of the tile sees every key of key tile j?
       const bool full_tile = key0 + kBN - 1 <= P + qt0;
       if (!__all_sync(0xffffffffu,
-                      mbar_wait(smem_u32(&sm.s_full[t]), j & 1))) {
+                      mbar_wait(smem_u32(&sm.s_full[t][b]), (j >> 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float s[kBN];
+      tmem_ld64(s_addr + b * kBN, s);
       const uint32_t bad = sm.bad_pages[st];
-      const bool plain = full_tile && bad == 0;
-
-      // ---- pass 1: row maximum of the raw scores ------------------------------
-      float mx = -INFINITY;
+      if (!(full_tile && bad == 0)) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float s[64];
-        tmem_ld64(s_addr + h * 64, s);
-        if (plain) {
-#pragma unroll
-          for (int x = 0; x < 64; x += 2) mx = fmax3(mx, s[x], s[x + 1]);
-        } else {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) {
-            const int key = key0 + h * 64 + x;
-            const bool vis =
-                key <= limit && !((bad >> ((h * 64 + x) / kPS)) & 1u);
-            mx = fmaxf(mx, vis ? s[x] : -INFINITY);
-          }
+        for (int x = 0; x < kBN; ++x) {
+          const int key = key0 + x;
+          const bool vis = key <= limit && !((bad >> (x / kPS)) & 1u);
+          s[x] = vis ? s[x] : -INFINITY;
         }
       }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int x = 0; x < kBN; x += 2) mx = fmax3(mx, s[x], s[x + 1]);
       const float m_tile = mx * c;   // scale > 0, so max commutes with it
-
-      // ---- P.V of the previous tile must be done before P is overwritten -------
-      if (j >= 1 &&
-          !__all_sync(0xffffffffu,
-                      mbar_wait(smem_u32(&sm.o_full[t]), (j - 1) & 1))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
 
       // ---- lazy rescale: move the running max only when it grows > 2^8 ----------
       const bool grow = m_tile > m_run + kRescaleThreshold;
@@ -324,7 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = fast_exp2(m_run - m_new);   // 0 when m_run = -inf
         l_run *= alpha;
         m_run = m_new;
-        if (j >= 1) {   // O holds the earlier tiles: rescale it in place
+        if (j >= 1) {   // O holds tiles < j once P.V of tile j-1 is done
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(smem_u32(&sm.o_done[t][(j - 1) & 1]),
+                                    ((j - 1) >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           float o[64];
           tmem_ld64(o_addr, o);
 #pragma unroll
@@ -334,47 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
 
-      // ---- pass 2: exponentials, row sum, P_hi / P_lo into shared memory --------
+      // ---- exponentials, row sum, P_hi / P_lo back into the S columns ------------
       float lsum = 0.f;
+      uint32_t hi[kBN / 2], lo[kBN / 2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float s[64];
-        tmem_ld64(s_addr + h * 64, s);
-        if (plain) {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) s[x] = fast_exp2(fmaf(s[x], c, -m_use));
-        } else {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) {
-            const int key = key0 + h * 64 + x;
-            const bool vis =
-                key <= limit && !((bad >> ((h * 64 + x) / kPS)) & 1u);
-            s[x] = vis ? fast_exp2(fmaf(s[x], c, -m_use)) : 0.f;
-          }
-        }
-        uint8_t* phi = sm.p[t][0][h] + r * kRowBytes;
-        uint8_t* plo = sm.p[t][1][h] + r * kRowBytes;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = s[ch * 8 + 2 * e], x1 = s[ch * 8 + 2 * e + 1];
-            lsum += x0 + x1;
-            hi[e] = pack_bf16x2(x0, x1);
-            lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
-          }
-          const int off = (ch ^ (r & 7)) * 16;
-          *reinterpret_cast<uint4*>(phi + off) =
-              make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(plo + off) =
-              make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
+      for (int e = 0; e < kBN / 2; ++e) {
+        const float x0 = fast_exp2(fmaf(s[2 * e], c, -m_use));
+        const float x1 = fast_exp2(fmaf(s[2 * e + 1], c, -m_use));
+        lsum += x0 + x1;
+        hi[e] = pack_bf16x2(x0, x1);
+        lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
       }
+      tmem_st32(s_addr + b * kBN, hi);
+      tmem_st32(s_addr + b * kBN + kBN / 2, lo);
       l_run += lsum;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[t]));
 
       // ---- keys past the context in a loaded page may hold stale data: zero
       //      their V rows (once per key tile, by the query tile whose P.V on
@@ -390,16 +365,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(0, 0, 0, 0);
         }
       }
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();   // the zeroed V rows, for the MMA
+      tc_fence_before();          // the P stores, for the MMA
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[t]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[t][b]));
     }
 
     // ---- wait for the last P.V, normalise and store --------------------------------
     float o[64];
     if (ok && my_tiles > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_full[t]),
-                                          (my_tiles - 1) & 1))) {
+        __all_sync(0xffffffffu,
+                   mbar_wait(smem_u32(&sm.o_done[t][(my_tiles - 1) & 1]),
+                             ((my_tiles - 1) >> 1) & 1))) {
       tc_fence_after();
       tmem_ld64(o_addr, o);
     } else {
