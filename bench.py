@@ -5,15 +5,26 @@
                     [--workload llama|mix|long|prefill|tiny]
 
 A step is one pass of the hot path over one batch:
-  llama / mix / tiny : the decode step -- append one token per sequence and
-                       attend over the whole paged context -- as the single
-                       fused launch tv_paged_decode_append (--unfused: the
-                       two calls tv_kv_append + tv_paged_decode);
+  llama / tiny       : the decode step -- append one token per sequence and
+                       attend over the whole paged context -- as one launch
+                       of tv_paged_decode_append (one CTA per sequence and KV
+                       head: equal lengths fill the GPU evenly);
+  mix                : the same step as one launch of tv_paged_decode_balanced
+                       with k_new/v_new (the work-balanced grid: mixed lengths
+                       would leave the one-CTA-per-pair grid with a long
+                       tail);
+                       --balanced / --per-pair pick either kernel for any
+                       decode workload, --unfused runs tv_kv_append +
+                       tv_paged_decode;
   long               : tv_kv_append, tv_paged_decode_split (512-token
                        partitions), tv_split_merge;
   prefill            : tv_kv_append of the 512-token chunks, then
                        tv_paged_prefill on the tensor cores.
 The default is the Llama-3.2-1B-shaped decode (64 sequences x 2048 tokens).
+Single-launch steps are timed as CUDA-graph replays of the K steps (chunks
+of up to 200 launches, back to back on one stream; --eager: one host launch
+per step with events around it); the end-to-end leg always launches from
+the host through the C ABI.
 Under torchrun every rank runs its own replica of the batch (sequences are
 independent; no collective touches the data path) and the whole-job value
 is the units of all ranks over the slowest rank's device time.
@@ -82,15 +93,27 @@ def _workload(name):
             "tiny": W.tiny_decode}[name]()
 
 
-def _config(wl, name, unfused=False):
+def _default_kind(name):
+    return {"prefill": "prefill", "long": "split",
+            "mix": "balanced"}.get(name, "fused")
+
+
+def _config(wl, name, kind=None):
+    kind = kind or _default_kind(name)
     cfg = {"workload": wl.name, "batch": wl.num_seqs,
            "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
            "head_dim": wl.head_dim, "page_size": wl.page_size,
            "num_pages": wl.num_pages,
            "context_tokens": int(wl.context_lens.sum())}
     if name in ("llama", "mix", "tiny"):
-        cfg["step"] = ("tv_kv_append + tv_paged_decode" if unfused else
-                       "tv_paged_decode_append (fused append + decode)")
+        cfg["step"] = {
+            "decode": "tv_kv_append + tv_paged_decode",
+            "fused": "tv_paged_decode_append (fused append + decode, one "
+                     "CTA per sequence and KV head)",
+            "split": "tv_kv_append + tv_paged_decode_split + "
+                     "tv_split_merge",
+        }.get(kind, "tv_paged_decode_balanced (fused append + decode, "
+                    "work-balanced persistent grid)")
     elif name == "long":
         cfg["step"] = ("tv_kv_append + tv_paged_decode_split + "
                        "tv_split_merge")
@@ -166,7 +189,8 @@ class TVRunner:
     """Device buffers and the calls of one step, marshalled once so that the
     host submits a step in a few microseconds."""
 
-    def __init__(self, wl, name, device, unfused=False, split_tokens=0):
+    def __init__(self, wl, name, device, unfused=False, split_tokens=0,
+                 per_pair=False, balanced=False):
         import torch
         from paged_kv_cache_376_b200 import _lib
         from paged_kv_cache_376_b200.device import upload
@@ -177,7 +201,12 @@ class TVRunner:
         self.out = torch.empty_like(db.q)
         self.kind = ("prefill" if name == "prefill" else
                      "split" if name == "long" or split_tokens else
-                     "decode" if unfused else "fused")
+                     "decode" if unfused else
+                     "fused" if per_pair else
+                     "balanced" if balanced else _default_kind(name))
+        if self.kind == "balanced":
+            self.ws = _lib.decode_workspace(wl.num_seqs, wl.num_q_heads,
+                                            wl.num_kv_heads, device)
         if self.kind == "split":
             if split_tokens:
                 wl.partition_tokens = split_tokens
@@ -203,6 +232,19 @@ class TVRunner:
         num_pages, ps, hkv, d = db.k_pool.shape
         b, hq = db.context_lens.shape[0], db.q.shape[1]
         mb = db.block_tables.shape[1]
+        if self.kind == "balanced":
+            if timing is not None:
+                timing[0].record(self.stream)
+            st = lib.tv_paged_decode_balanced(
+                self._p(self.out), self._p(db.q), self._p(db.k_new),
+                self._p(db.v_new), self._p(db.k_pool), self._p(db.v_pool),
+                self._p(db.block_tables), mb, self._p(db.context_lens), b, hq,
+                hkv, d, ps, num_pages, wl.scale, self._p(self.ws),
+                self.ws.numel(), self._p(db.err), s)
+            assert st == 0, st
+            if timing is not None:
+                timing[1].record(self.stream)
+            return
         if self.kind == "fused":
             if timing is not None:
                 timing[0].record(self.stream)
@@ -253,7 +295,32 @@ class TVRunner:
             assert st == 0, st
 
     def launches_per_step(self):
-        return {"split": 3, "fused": 1}.get(self.kind, 2)
+        return {"split": 3, "fused": 1, "balanced": 1}.get(self.kind, 2)
+
+    def graphs(self, steps, chunk=200):
+        """CUDA graphs that replay exactly ``steps`` steps: a list of
+        graphs, each captured from ``chunk`` (or fewer) consecutive steps."""
+        torch = self.torch
+        cap = torch.cuda.Stream(self.device)
+        cap.wait_stream(torch.cuda.current_stream(self.device))
+        home, self.stream = self.stream, cap
+        made, plan = {}, []
+        try:
+            left = steps
+            while left:
+                n = min(chunk, left)
+                if n not in made:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=cap):
+                        for _ in range(n):
+                            self.step()
+                    made[n] = g
+                plan.append(made[n])
+                left -= n
+        finally:
+            self.stream = home
+        torch.cuda.current_stream(self.device).wait_stream(cap)
+        return plan
 
     # -- end to end: host inputs in, host result out, through the C ABI ------
     def setup_e2e(self):
@@ -301,7 +368,9 @@ def run_tv(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     wl = _workload(args.workload)
     runner = TVRunner(wl, args.workload, device, unfused=args.unfused,
-                      split_tokens=args.split_tokens)
+                      split_tokens=args.split_tokens, per_pair=args.per_pair,
+                      balanced=args.balanced)
+    use_graph = (runner.launches_per_step() == 1 and not args.eager)
     per_step, unit, seqs = _units(wl, args.workload)
     hbm, tfl, tfl_sus, peak_src = _peaks()
     K, Wm = args.steps, args.warmup
@@ -313,6 +382,9 @@ def run_tv(args, rank, world, local_rank):
 
     for _ in range(Wm):
         runner.step()
+    plan = runner.graphs(K) if use_graph else None
+    if plan:
+        plan[0].replay()          # untimed: uploads the graph
     barrier()
 
     # ---- device-timed region ------------------------------------------------
@@ -328,14 +400,20 @@ def run_tv(args, rank, world, local_rank):
     barrier()
     wall0 = time.perf_counter()
     t0.record()
-    for i in range(K):
-        runner.step(ev[i])
+    if plan:
+        for g in plan:
+            g.replay()
+    else:
+        for i in range(K):
+            runner.step(ev[i])
     t1.record()
     barrier()
     wall = time.perf_counter() - wall0
     clock_info = clocks.stop() if clocks else None
     ms = t0.elapsed_time(t1)
-    kern_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    # one launch per step under a graph: the kernel's share is the step
+    kern_ms = (ms / K if plan else
+               statistics.fmean(a.elapsed_time(b) for a, b in ev))
     ms_max = _max_over_ranks(ms, world, device)
     kern_ms_max = _max_over_ranks(kern_ms, world, device)
     err = int(runner.db.err.item())
@@ -360,7 +438,8 @@ def run_tv(args, rank, world, local_rank):
     kern_per_launch = per_step / (kern_ms_max / 1e3)     # GB/s or TFLOP/s
     kernel_name = {"decode": "tv_paged_decode", "split":
                    "tv_paged_decode_split", "prefill": "tv_paged_prefill",
-                   "fused": "tv_paged_decode_append"}[runner.kind]
+                   "fused": "tv_paged_decode_append",
+                   "balanced": "tv_paged_decode_balanced"}[runner.kind]
     if unit == "GB/s":
         peak, bound, src = hbm, "hbm", peak_src
     else:
@@ -373,9 +452,12 @@ def run_tv(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, shuffled "
         "page pool)",
-        "config": dict(_config(wl, args.workload, args.unfused),
+        "config": dict(_config(wl, args.workload, runner.kind),
                        parallelism=f"replicas{world}" if world > 1
-                       else "single GPU"),
+                       else "single GPU",
+                       launch=("CUDA graphs of up to 200 steps, replayed "
+                               "back to back" if plan else
+                               "one host launch per step")),
         "seq_steps_per_s": round(whole_job_rate(seqs, K, ms_max, world), 1),
         "hbm_frac" if unit == "GB/s" else "tensor_frac":
             round(value / world / peak, 4),
@@ -559,6 +641,14 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="decode step as tv_kv_append + tv_paged_decode")
+    ap.add_argument("--per-pair", action="store_true",
+                    help="decode step as tv_paged_decode_append (one CTA "
+                         "per sequence and KV head)")
+    ap.add_argument("--balanced", action="store_true",
+                    help="decode step as tv_paged_decode_balanced (the "
+                         "work-balanced grid) with the append fused")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every timed step from the host (no graph)")
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="decode step as tv_kv_append + tv_paged_decode_split "
                          "(partitions of this many tokens) + tv_split_merge")

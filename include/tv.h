@@ -53,6 +53,7 @@
 #ifndef TV_H_
 #define TV_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -150,6 +151,55 @@ tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
                                  int head_dim, int page_size,
                                  int64_t num_pages, float scale,
                                  uint32_t* err, void* stream);
+
+/*
+ * tv_decode_workspace_size -- bytes of device workspace that
+ * tv_paged_decode_balanced needs for up to num_seqs sequences on the
+ * current device (it depends on the device's SM count).
+ *   bytes   host pointer, written on TV_OK
+ */
+tv_status tv_decode_workspace_size(int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim,
+                                   size_t* bytes);
+
+/*
+ * tv_paged_decode_balanced -- the result of tv_paged_decode (k_new == NULL)
+ * or of tv_paged_decode_append (k_new, v_new given), computed by a
+ * persistent grid that gives every warp the same number of K/V pages: the
+ * pages of all (sequence, KV head) pairs are laid end to end and cut into
+ * equal contiguous ranges.  A pair cut by range boundaries is finished from
+ * per-warp partials (running max, sum and weighted V sum of each head) by
+ * the log-sum-exp rule of tv_split_merge ([P1] "在线Softmax": partial
+ * softmax results combine exactly through their maxima and sums); the warp
+ * that writes the last partial of a pair merges them.  The source pages
+ * give no schedule; this one removes the idle SMs that a grid of one CTA
+ * per pair leaves when the pair count is not a multiple of the resident
+ * CTA slots, and the tail that mixed context lengths cause.
+ *   workspace        device memory of at least tv_decode_workspace_size()
+ *                    bytes, 16-byte aligned, ZERO-FILLED before its first
+ *                    use; each call leaves it zero-filled again unless a
+ *                    bounded wait ran out (TV_DEVERR_TIMEOUT), after which
+ *                    it must be zero-filled again
+ *   workspace_bytes  its size; too small returns TV_ERR_INVALID_ARG
+ *   other arguments as tv_paged_decode / tv_paged_decode_append.
+ * Calls that overlap on the GPU (unordered streams) need separate
+ * workspaces.  Above 512 sequences, with max_blocks_per_seq >= 2^24 or
+ * num_pages >= 2^26 - 1, or when num_seqs * num_kv_heads *
+ * max_blocks_per_seq reaches 2^31, the call runs the one-CTA-per-pair
+ * kernel of tv_paged_decode instead and leaves the workspace untouched.
+ * Results equal tv_paged_decode's up to fp32 summation order.
+ */
+tv_status tv_paged_decode_balanced(void* out, const void* q,
+                                   const void* k_new, const void* v_new,
+                                   void* k_pool, void* v_pool,
+                                   const int32_t* block_tables,
+                                   int max_blocks_per_seq,
+                                   const int32_t* context_lens, int num_seqs,
+                                   int num_q_heads, int num_kv_heads,
+                                   int head_dim, int page_size,
+                                   int64_t num_pages, float scale,
+                                   void* workspace, size_t workspace_bytes,
+                                   uint32_t* err, void* stream);
 
 /*
  * tv_paged_decode_split -- tv_paged_decode restricted to logical key

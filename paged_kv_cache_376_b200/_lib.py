@@ -47,6 +47,11 @@ SIGNATURES = {
     "tv_paged_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I,
                                           _I, _I, _I, _I64, _F, _I, _I, _P,
                                           _P]),
+    "tv_decode_workspace_size": (_I, [_I, _I, _I, _I,
+                                      ctypes.POINTER(ctypes.c_size_t)]),
+    "tv_paged_decode_balanced": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
+                                      _I, _I, _I, _I, _I64, _F, _P,
+                                      ctypes.c_size_t, _P, _P]),
 }
 
 _lib = None
@@ -278,3 +283,56 @@ def tv_paged_decode_split_static(out, q, k_pool, v_pool, block_tables,
         block_tables.shape[1], _ptr(context_lens), b, hq, hkv, d, page_size,
         num_pages, float(scale), int(partition_tokens), int(max_partitions),
         _ptr(err), _stream(stream)), "tv_paged_decode_split_static")
+
+
+def tv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                             head_dim=64):
+    """Bytes of workspace tv_paged_decode_balanced needs on the current
+    device for up to num_seqs sequences."""
+    lib = load()
+    out = ctypes.c_size_t(0)
+    _check(lib.tv_decode_workspace_size(int(num_seqs), int(num_q_heads),
+                                        int(num_kv_heads), int(head_dim),
+                                        ctypes.byref(out)),
+           "tv_decode_workspace_size")
+    return out.value
+
+
+def decode_workspace(num_seqs, num_q_heads, num_kv_heads, device=None):
+    """A zero-filled uint8 workspace of the size tv_decode_workspace_size
+    gives (the balanced decode leaves it zero-filled after every call)."""
+    n = tv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def tv_paged_decode_balanced(out, q, k_pool, v_pool, block_tables,
+                             context_lens, scale, workspace, k_new=None,
+                             v_new=None, err=None, stream=None):
+    """Work-balanced decode (fused with the append when k_new/v_new are
+    given): out[B][Hq][D] as tv_paged_decode / tv_paged_decode_append."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_pool", k_pool),
+                 ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        _cuda(k_new, bf, "k_new"), _cuda(v_new, bf, "v_new")
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    _cuda(workspace, torch.uint8, "workspace")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != b or (
+            k_new is not None and (k_new.shape != (b, hkv, d) or
+                                   v_new.shape != k_new.shape)):
+        raise ValueError("shape mismatch")
+    _check(lib.tv_paged_decode_balanced(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+        _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), b, hq, hkv, d, page_size, num_pages, float(scale),
+        _ptr(workspace), workspace.numel(), _ptr(err), _stream(stream)),
+        "tv_paged_decode_balanced")

@@ -31,6 +31,7 @@
 //    owns the page holding position context_len-1 writes the new token's row
 //    of its KV head into the pool and into its staged copy of that page, so
 //    the step is one launch and the new row is never read back from HBM.
+#include "tv_decode.cuh"
 #include "tv_device.cuh"
 #include "tv_kernels.h"
 
@@ -44,6 +45,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kRowBytes = kD * 2;                 // one token, one KV head
 constexpr int kSliceBytes = kPS * kRowBytes;      // 2 KB
 constexpr int kStageBytes = 2 * kSliceBytes;      // K slice + V slice
+constexpr float kLazy = 8.f;   // log2 of the growth the running sums allow
 
 template <int kStages>
 struct DecodeSmem {
@@ -125,12 +127,15 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
   // ---- q for the G heads of this KV head, pre-scaled by scale*log2(e) -----
   // Element pairs (2i, 2i+1) of this lane's 8-element chunk, as float2 so
-  // the dot products run on the packed fp32x2 FMA pipe.
+  // the dot products run on the packed fp32x2 FMA pipe.  Position h holds
+  // head h ^ rs_mask (the order reduce_scatter8 expects).
+  const int qmask = rs_mask<G>(chk);
   float2 q2[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const uint4 v = *reinterpret_cast<const uint4*>(
-        a.q + ((size_t)seq * a.num_q_heads + kvh * G + h) * kD + chk * 8);
+        a.q + ((size_t)seq * a.num_q_heads + kvh * G + (h ^ qmask)) * kD +
+        chk * 8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -181,9 +186,14 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   bool failed = false;
   int issued = min(my_n, kStages);
   int i = 0;
-  for (; i < my_n; ++i) {
-    const int stage = i % kStages;
-    const uint32_t parity = (i / kStages) & 1;
+  // kStages pages per outer step, unrolled, so each page's ring slot and
+  // barrier address are constants.
+  uint32_t parity = 0;
+  for (int i0 = 0; i0 < my_n; i0 += kStages, parity ^= 1) {
+#pragma unroll
+  for (int stage = 0; stage < kStages; ++stage) {
+    i = i0 + stage;
+    if (i >= my_n) break;
     if ((i & 31) == 0 && i > 0) {
       pid_cur = pid_next;
       pid_next = load_pids((i >> 5) + 1);
@@ -201,8 +211,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       failed = true;
       break;
     }
-    const uint8_t* kbase = &sm.ring[warp][stage][0];
-    const uint8_t* vbase = kbase + kSliceBytes;
+    uint8_t* kbase = &sm.ring[warp][stage][0];
+    uint8_t* vbase = kbase + kSliceBytes;
     if (kAppend && i == app_i) {
       // the staged page now gets the new row; the pool keeps it for later
       if (page_ok && lane < 16) {
@@ -215,6 +225,16 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
             chk * 8) = app_row;
       }
       __syncwarp();
+    }
+    if (!full_page) {
+      // Rows past the range (or the whole of a bad page) get p = 0; zero
+      // their V so that 0 * a stale NaN never reaches the sum.  Each lane
+      // clears exactly the rows and chunk it reads below.
+#pragma unroll
+      for (int r = grp; r < kPS; r += 4)
+        if (!(page_ok && page_tok0 + r < tok_end))
+          *reinterpret_cast<uint4*>(vbase + r * kRowBytes + chk * 16) =
+              make_uint4(0, 0, 0, 0);
     }
 
     // ---- scores: token it*4+grp, head my_head ---------------------------------
@@ -236,39 +256,23 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
         for (int t = 1; t < 4; ++t) d2 = __ffma2_rn(q2[h][t], k2[t], d2);
         part[h] = d2.x + d2.y;
       }
-      // reduce-scatter over the 8 lanes of the group: at each xor step a
-      // lane keeps half of its values and adds the partner's copy of them
-      int n = G;
-#pragma unroll
-      for (int off = 4; off >= 1; off >>= 1) {
-        if (n > 1) {
-          const bool upper = (chk & off) != 0;
-#pragma unroll
-          for (int h = 0; h < G / 2; ++h) {
-            if (h < n / 2) {
-              const float keep = upper ? part[h + n / 2] : part[h];
-              const float send = upper ? part[h] : part[h + n / 2];
-              part[h] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-            }
-          }
-          n >>= 1;
-        } else {
-          part[0] += __shfl_xor_sync(0xffffffffu, part[0], off);
-        }
-      }
-      s[it] = part[0];
+      // reduce-scatter over the 8 lanes of the group (no selects: the q
+      // positions are permuted per lane)
+      s[it] = reduce_scatter8<G>(part);
       if (!full_page) {
         const bool valid = page_ok && (page_tok0 + r) < tok_end;
         s[it] = valid ? s[it] : -INFINITY;
       }
     }
 
-    // ---- online softmax, once per page -----------------------------------------
+    // ---- online softmax, once per page, with a lazy offset -----------------------
+    // The offset m_run only moves when a page maximum exceeds it by more
+    // than 2^kLazy (base 2): exp2(s - m_run) then stays below 2^kLazy, and
+    // any offset gives the same acc / l.
     float pm = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
     pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
     pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
-    if (__any_sync(0xffffffffu, pm > m_run)) {
-      // the running max moved for some head: rescale (rare after warm-up)
+    if (__any_sync(0xffffffffu, pm > m_run + kLazy)) {
       const float m_new = fmaxf(m_run, pm);
       const float alpha = fast_exp2(m_run - (m_new == -INFINITY ? 0.f : m_new));
       m_run = m_new;
@@ -289,12 +293,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       const int r = it * 4 + grp;
       const float p = fast_exp2(s[it] - m_use);
       l_run += p;
-      uint4 vv =
+      const uint4 vv =
           *reinterpret_cast<const uint4*>(vbase + r * kRowBytes + chk * 16);
-      if (!full_page) {
-        const bool valid = page_ok && (page_tok0 + r) < tok_end;
-        if (!valid) vv = make_uint4(0, 0, 0, 0);  // stale slots may be NaN
-      }
       const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
       float2 v2[4];
 #pragma unroll
@@ -318,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       if (lane == 0) issue(pid_j, stage);
       ++issued;
     }
+  }
+  if (failed) break;
   }
 
   if (failed) {

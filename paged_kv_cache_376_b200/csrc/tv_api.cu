@@ -55,7 +55,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // The pool seen as a 2-D bf16 tensor [num_pages * page_size][Hkv * D]; the
-// box is one page of one KV head: 16 rows x 64 elements (128 B).
+// box is one page of one KV head: 16 rows x 64 elements (128 B).  The 256-byte
+// L2 promotion also fetches the neighbouring KV head's row; every decode grid
+// reads the KV heads of a page at about the same time, so that row is an L2
+// hit for its reader, not a second DRAM read.
 tv_status pool_tensor_map(CUtensorMap* map, const void* pool,
                           int64_t num_pages, int num_kv_heads,
                           CUtensorMapSwizzle swizzle) {
@@ -151,6 +154,36 @@ tv_status tv_kv_append(const void* k_new, const void* v_new,
       static_cast<cudaStream_t>(stream)));
 }
 
+// Device workspace of the work-balanced decode: per-item counters, then two
+// partial-result slots per warp of the persistent grid.
+struct BalancedWorkspace {
+  void* base;
+  size_t bytes;
+};
+
+static int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return 0;
+  return sms;
+}
+
+static size_t counters_bytes(int num_seqs, int num_kv_heads) {
+  return ((size_t)num_seqs * num_kv_heads * 4 + 255) / 256 * 256;
+}
+
+static int balanced_ctas(int group) {
+  const int a = tv::balanced_decode_ctas_per_sm(group, false);
+  const int b = tv::balanced_decode_ctas_per_sm(group, true);
+  return device_sms() * (a > b ? a : b);
+}
+
+static size_t partials_bytes(int ctas) {
+  return (size_t)ctas * 4 * 2 * tv::kSlotFloats * sizeof(float);
+}
+
 static tv_status decode_common(void* out, float* partial_out,
                                float* partial_lse, const void* q,
                                const void* k_new, const void* v_new,
@@ -161,7 +194,8 @@ static tv_status decode_common(void* out, float* partial_out,
                                int num_q_heads, int num_kv_heads, int head_dim,
                                int page_size, int64_t num_pages, float scale,
                                int partition_tokens, int max_partitions,
-                               bool split, uint32_t* err, void* stream) {
+                               bool split, uint32_t* err, void* stream,
+                               const BalancedWorkspace* ws = nullptr) {
   tv_status st =
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
   if (st != TV_OK) return st;
@@ -187,6 +221,11 @@ static tv_status decode_common(void* out, float* partial_out,
   if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
     return TV_ERR_INVALID_ARG;
 
+  const bool balanced = ws && num_seqs <= tv::kMaxBalancedSeqs &&
+                        max_blocks_per_seq < (1 << 24) &&
+                        num_pages < (1 << 26) - 1 &&
+                        (int64_t)num_seqs * num_kv_heads *
+                                max_blocks_per_seq < INT32_MAX;
   CUtensorMap tk, tvm;
   st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -213,8 +252,34 @@ static tv_status decode_common(void* out, float* partial_out,
   a.partition_tokens = split ? partition_tokens : 0;
   a.max_partitions = split ? max_partitions : 1;
   a.scale_log2 = scale * 1.4426950408889634f;
+  const int group = num_q_heads / num_kv_heads;
+  // The balanced grid needs the prefix sums of every sequence in shared
+  // memory, all flattened page positions in int32, page indices in 24 bits
+  // and physical page ids in 26 bits (the condition `balanced` above);
+  // beyond that the
+  // one-CTA-per-(sequence, KV head) kernel serves the call.
+  if (balanced) {
+    const int cap = balanced_ctas(group);
+    if (cap <= 0) return cuda_status(cudaErrorUnknown);
+    const size_t cb = counters_bytes(num_seqs, num_kv_heads);
+    if (ws->bytes < cb + partials_bytes(cap)) return TV_ERR_INVALID_ARG;
+    // groups of num_kv_heads warps, each with >= kMinPagesPerWarp pages
+    // (num_seqs * max_blocks_per_seq bounds the page count from above)
+    const int64_t groups = ((int64_t)num_seqs * max_blocks_per_seq +
+                            tv::kMinPagesPerWarp - 1) / tv::kMinPagesPerWarp;
+    const int64_t want = (groups * num_kv_heads + 3) / 4;
+    const int64_t least = (num_kv_heads + 3) / 4;   // one whole group
+    if (cap < least) return TV_ERR_UNSUPPORTED;
+    const int ctas = (int)(want < least ? least : (want < cap ? want : cap));
+    a.num_seqs = num_seqs;
+    a.num_kv_heads = num_kv_heads;
+    a.ws_counters = static_cast<int32_t*>(ws->base);
+    a.ws_partials = reinterpret_cast<float*>(static_cast<char*>(ws->base) + cb);
+    return cuda_status(tv::launch_balanced_decode(
+        a, tk, tvm, group, ctas, static_cast<cudaStream_t>(stream)));
+  }
   return cuda_status(tv::launch_paged_decode(
-      a, tk, tvm, num_kv_heads, num_seqs, num_q_heads / num_kv_heads, split,
+      a, tk, tvm, num_kv_heads, num_seqs, group, split,
       split ? max_partitions : 1, static_cast<cudaStream_t>(stream)));
 }
 
@@ -244,6 +309,41 @@ tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
                        block_tables, max_blocks_per_seq, context_lens,
                        num_seqs, num_q_heads, num_kv_heads, head_dim,
                        page_size, num_pages, scale, 0, 1, false, err, stream);
+}
+
+tv_status tv_decode_workspace_size(int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim,
+                                   size_t* bytes) {
+  if (!bytes) return TV_ERR_INVALID_ARG;
+  tv_status st =
+      check_attention_shape(num_q_heads, num_kv_heads, head_dim, kPageSize);
+  if (st != TV_OK) return st;
+  if (num_seqs < 0) return TV_ERR_INVALID_ARG;
+  const int cap = balanced_ctas(num_q_heads / num_kv_heads);
+  if (cap <= 0) return cuda_status(cudaErrorUnknown);
+  *bytes = counters_bytes(num_seqs, num_kv_heads) + partials_bytes(cap);
+  return TV_OK;
+}
+
+tv_status tv_paged_decode_balanced(void* out, const void* q,
+                                   const void* k_new, const void* v_new,
+                                   void* k_pool, void* v_pool,
+                                   const int32_t* block_tables,
+                                   int max_blocks_per_seq,
+                                   const int32_t* context_lens, int num_seqs,
+                                   int num_q_heads, int num_kv_heads,
+                                   int head_dim, int page_size,
+                                   int64_t num_pages, float scale,
+                                   void* workspace, size_t workspace_bytes,
+                                   uint32_t* err, void* stream) {
+  if (num_seqs > 0 && (!workspace || !aligned16(workspace)))
+    return TV_ERR_INVALID_ARG;
+  const BalancedWorkspace ws{workspace, workspace_bytes};
+  return decode_common(out, nullptr, nullptr, q, k_new, v_new, k_pool, v_pool,
+                       block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, 0, 1, false, err, stream,
+                       &ws);
 }
 
 tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,

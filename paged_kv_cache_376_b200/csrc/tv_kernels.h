@@ -26,7 +26,22 @@ struct DecodeArgs {
   int partition_tokens;
   int max_partitions;
   float scale_log2;              // scale * log2(e)
+  // work-balanced decode only
+  int num_seqs;
+  int num_kv_heads;
+  int32_t* ws_counters;          // [B * Hkv], zero between launches
+  float* ws_partials;            // [warps][2][kSlotFloats]
 };
+
+// Work-balanced decode (paged_decode_balanced.cu).
+constexpr int kMaxBalancedSeqs = 512;    // prefix sums live in shared memory
+constexpr int kMinPagesPerWarp = 4;      // smallest range a warp is given
+constexpr int kSlotFloats = 16 + 8 * 64; // m[8], l[8], acc[8][64] per segment
+
+int balanced_decode_ctas_per_sm(int group, bool append);
+cudaError_t launch_balanced_decode(const DecodeArgs& a, const CUtensorMap& tk,
+                                   const CUtensorMap& tv, int group, int ctas,
+                                   cudaStream_t stream);
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
                                 const CUtensorMap& tv, int num_kv_heads,
