@@ -186,14 +186,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   bool failed = false;
   int issued = min(my_n, kStages);
   int i = 0;
-  // kStages pages per outer step, unrolled, so each page's ring slot and
-  // barrier address are constants.
-  uint32_t parity = 0;
-  for (int i0 = 0; i0 < my_n; i0 += kStages, parity ^= 1) {
-#pragma unroll
-  for (int stage = 0; stage < kStages; ++stage) {
-    i = i0 + stage;
-    if (i >= my_n) break;
+  for (; i < my_n; ++i) {
+    const int stage = i % kStages;
+    const uint32_t parity = (i / kStages) & 1;
     if ((i & 31) == 0 && i > 0) {
       pid_cur = pid_next;
       pid_next = load_pids((i >> 5) + 1);
@@ -318,8 +313,6 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       if (lane == 0) issue(pid_j, stage);
       ++issued;
     }
-  }
-  if (failed) break;
   }
 
   if (failed) {
