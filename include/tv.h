@@ -46,6 +46,9 @@
  *       TV_DEVERR_TIMEOUT      a bounded internal wait (2 s) ran out; the
  *                              affected outputs are zeros
  *       TV_DEVERR_BAD_QUERY    query_start_loc inconsistent with the context
+ *       TV_DEVERR_POOL_EMPTY   the page pool had too few free pages for a
+ *                              sequence (tv_pool_append_slots)
+ *       TV_DEVERR_BAD_SEQ      a fork or release named a bad sequence
  *   - Outputs must not alias inputs.
  *   - Return: TV_OK, or an error status; TV_ERR_CUDA means the launch failed
  *     (tv_last_cuda_error() gives the CUDA error code).
@@ -74,7 +77,9 @@ enum {
   TV_DEVERR_BAD_PAGE = 1u << 1,
   TV_DEVERR_BAD_CONTEXT = 1u << 2,
   TV_DEVERR_TIMEOUT = 1u << 3,
-  TV_DEVERR_BAD_QUERY = 1u << 4
+  TV_DEVERR_BAD_QUERY = 1u << 4,
+  TV_DEVERR_POOL_EMPTY = 1u << 5,
+  TV_DEVERR_BAD_SEQ = 1u << 6
 };
 
 /* Human-readable name of a status. Never NULL. */
@@ -300,6 +305,118 @@ tv_status tv_paged_decode_split_static(
     int num_kv_heads, int head_dim, int page_size, int64_t num_pages,
     float scale, int partition_tokens, int max_partitions, uint32_t* err,
     void* stream);
+
+/*
+ * ---- Device page pool -------------------------------------------------------
+ * The KV pages of [P3] "内存池管理" as a device-resident pool: a free-page stack
+ * and a reference count per page, so that a decode step -- room for the new
+ * token, then tv_paged_decode_append -- needs no host round trip and can be
+ * captured in a CUDA graph.  Pages are allocated on demand, returned when a
+ * sequence is released, and shared between sequences by tv_pool_fork (prefix
+ * sharing); a shared page is copied before it is written ([P1]
+ * "PagedAttention": copy-on-write).  The pages give no free-list layout, no
+ * order of allocation and no sharing rule beyond these; the rules below are
+ * this library's, chosen so every call is deterministic.
+ *
+ * pool_state: device int32 array of TV_POOL_STATE_INTS(num_pages) entries,
+ * caller-owned, set up by tv_pool_init and changed only by the tv_pool_*
+ * calls:
+ *   [0] number of free pages (top of the stack)   [2] slots written by the
+ *   last tv_pool_append_slots   [4 .. 4+NP) free-page stack (pop takes entry
+ *   top-1)   then NP reference counts and 2 x NP scratch words.
+ * A page's reference count is the number of block-table rows holding it.
+ * Every pool call serves at most 1024 sequences (TV_ERR_UNSUPPORTED above),
+ * runs as one CTA, and is ordered with the caller's other work by `stream`.
+ */
+#define TV_POOL_STATE_INTS(num_pages) (4 + 4 * (int64_t)(num_pages))
+
+/*
+ * tv_pool_init -- every page free, except those the first
+ * ceil(context_lens[s] / 16) entries of each block-table row hold (counted);
+ * the free pages are stacked in descending id order, so a fresh pool hands
+ * out pages 0, 1, 2, ...  block_tables may be NULL (an empty pool).
+ */
+tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages,
+                       const int32_t* block_tables, int max_blocks_per_seq,
+                       const int32_t* context_lens, int num_seqs,
+                       uint32_t* err, void* stream);
+
+/*
+ * tv_pool_append_slots -- room for num_new_tokens[s] tokens at positions
+ * context_lens[s] .. context_lens[s] + n - 1 of every sequence, in batch
+ * order:
+ *   - if the partly filled page those positions start in is shared (count
+ *     > 1), the sequence first takes a fresh page and copies that page's K
+ *     and V into it (copy-on-write), unless every holder of the page writes
+ *     into it in this call and this sequence is the last of them in batch
+ *     order (it keeps the page);
+ *   - then it takes one fresh page per page boundary crossed;
+ *   - needs are reserved in batch order and served all-or-nothing: once a
+ *     sequence cannot be served, no later one is (TV_DEVERR_POOL_EMPTY; those
+ *     sequences are left unchanged);
+ *   - context_lens[s] += n for every served sequence.
+ *   num_new_tokens  [num_seqs] int32, or NULL: one token for every sequence
+ *                   with context_lens[s] > 0 (a decode step)
+ *   slot_mapping    NULL, or room for the sum of n: receives the slots of the
+ *                   new tokens of the served sequences in batch order (as
+ *                   tv_kv_append takes them); their count is pool_state[2]
+ *   k_pool, v_pool  the pools (copy-on-write copies whole pages)
+ */
+tv_status tv_pool_append_slots(int32_t* pool_state, int64_t num_pages,
+                               int32_t* block_tables, int max_blocks_per_seq,
+                               int32_t* context_lens,
+                               const int32_t* num_new_tokens, int num_seqs,
+                               int32_t* slot_mapping, void* k_pool,
+                               void* v_pool, int num_kv_heads, int head_dim,
+                               int page_size, uint32_t* err, void* stream);
+
+/*
+ * tv_pool_fork -- for i = 0 .. num_pairs-1 in order: the empty sequence
+ * dst_seqs[i] (context 0) takes the block-table entries and context of
+ * src_seqs[i]; each shared page's count grows by one.  A pair whose
+ * destination is not empty, or that names a bad index, is skipped and
+ * flagged TV_DEVERR_BAD_SEQ.  src_seqs, dst_seqs: device int32 arrays.
+ */
+tv_status tv_pool_fork(int32_t* pool_state, int64_t num_pages,
+                       int32_t* block_tables, int max_blocks_per_seq,
+                       int32_t* context_lens, int num_seqs,
+                       const int32_t* src_seqs, const int32_t* dst_seqs,
+                       int num_pairs, uint32_t* err, void* stream);
+
+/*
+ * tv_pool_release -- for each listed sequence (device int32 array, in
+ * order) every page reference is dropped, its row becomes -1 and its
+ * context 0; pages whose count reaches zero go back on the stack in
+ * ascending id order (so the largest of them is handed out first).
+ */
+tv_status tv_pool_release(int32_t* pool_state, int64_t num_pages,
+                          int32_t* block_tables, int max_blocks_per_seq,
+                          int32_t* context_lens, int num_seqs,
+                          const int32_t* seqs, int num_release, uint32_t* err,
+                          void* stream);
+
+/*
+ * tv_decode_step -- one decode step of every live sequence, device-side
+ * only: tv_pool_append_slots with num_new_tokens = NULL, then
+ * tv_paged_decode_append (the new token's K/V go to position ctx-1 of the
+ * grown context; out = attention of q over it), or, when workspace is not
+ * NULL, tv_paged_decode_balanced with k_new / v_new and that workspace (for
+ * batches of mixed lengths).  Sequences with context 0
+ * are idle: they append nothing and output zeros.  Two launches, no host
+ * synchronisation, so a run of steps can be captured in one CUDA graph.
+ * A sequence left unserved by an empty pool (TV_DEVERR_POOL_EMPTY) has its
+ * last cached row overwritten by this step's row: keep at least one free
+ * page per live sequence.  Arguments as tv_pool_append_slots and
+ * tv_paged_decode_append.
+ */
+tv_status tv_decode_step(int32_t* pool_state, int64_t num_pages, void* out,
+                         const void* q, const void* k_new, const void* v_new,
+                         void* k_pool, void* v_pool, int32_t* block_tables,
+                         int max_blocks_per_seq, int32_t* context_lens,
+                         int num_seqs, int num_q_heads, int num_kv_heads,
+                         int head_dim, int page_size, float scale,
+                         void* workspace, size_t workspace_bytes,
+                         uint32_t* err, void* stream);
 
 #ifdef __cplusplus
 }

@@ -26,6 +26,8 @@ DEVERR_BAD_PAGE = 1 << 1
 DEVERR_BAD_CONTEXT = 1 << 2
 DEVERR_TIMEOUT = 1 << 3
 DEVERR_BAD_QUERY = 1 << 4
+DEVERR_POOL_EMPTY = 1 << 5
+DEVERR_BAD_SEQ = 1 << 6
 
 # (name, restype, argtypes) of every symbol include/tv.h declares
 _P, _I, _I64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
@@ -52,6 +54,14 @@ SIGNATURES = {
     "tv_paged_decode_balanced": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
                                       _I, _I, _I, _I, _I64, _F, _P,
                                       ctypes.c_size_t, _P, _P]),
+    "tv_pool_init": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P]),
+    "tv_pool_append_slots": (_I, [_P, _I64, _P, _I, _P, _P, _I, _P, _P, _P,
+                                  _I, _I, _I, _P, _P]),
+    "tv_pool_fork": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P, _I, _P, _P]),
+    "tv_pool_release": (_I, [_P, _I64, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "tv_decode_step": (_I, [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
+                            _I, _I, _I, _I, _F, _P, ctypes.c_size_t, _P,
+                            _P]),
 }
 
 _lib = None
@@ -336,3 +346,125 @@ def tv_paged_decode_balanced(out, q, k_pool, v_pool, block_tables,
         _ptr(context_lens), b, hq, hkv, d, page_size, num_pages, float(scale),
         _ptr(workspace), workspace.numel(), _ptr(err), _stream(stream)),
         "tv_paged_decode_balanced")
+
+
+# ---- device page pool --------------------------------------------------------
+
+def pool_state_ints(num_pages):
+    """TV_POOL_STATE_INTS(num_pages) of include/tv.h."""
+    return 4 + 4 * int(num_pages)
+
+
+def pool_state(num_pages, device=None):
+    """An (uninitialised) pool state array for tv_pool_init."""
+    return torch.zeros(pool_state_ints(num_pages), dtype=torch.int32,
+                       device=device or "cuda")
+
+
+def _pool_tables(block_tables, context_lens):
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if block_tables.shape[0] != context_lens.shape[0]:
+        raise ValueError("block_tables and context_lens disagree on num_seqs")
+    return block_tables.shape[1], block_tables.shape[0]
+
+
+def _pool_pages(state):
+    _cuda(state, torch.int32, "pool_state")
+    n = state.numel() - 4
+    if n <= 0 or n % 4:
+        raise ValueError("pool_state must hold 4 + 4 * num_pages ints")
+    return n // 4
+
+
+def tv_pool_init(state, block_tables=None, context_lens=None, err=None,
+                 stream=None):
+    lib = load()
+    num_pages = _pool_pages(state)
+    mb, b = (_pool_tables(block_tables, context_lens)
+             if block_tables is not None else (0, 0))
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    _check(lib.tv_pool_init(_ptr(state), num_pages, _ptr(block_tables), mb,
+                            _ptr(context_lens), b, _ptr(err),
+                            _stream(stream)), "tv_pool_init")
+
+
+def tv_pool_append_slots(state, block_tables, context_lens, k_pool, v_pool,
+                         num_new_tokens=None, slot_mapping=None, err=None,
+                         stream=None):
+    lib = load()
+    num_pages = _pool_pages(state)
+    mb, b = _pool_tables(block_tables, context_lens)
+    _cuda(k_pool, torch.bfloat16, "k_pool"), _cuda(v_pool, torch.bfloat16,
+                                                   "v_pool")
+    if k_pool.shape[0] != num_pages:
+        raise ValueError("pool_state and k_pool disagree on num_pages")
+    for n, t in (("num_new_tokens", num_new_tokens),
+                 ("slot_mapping", slot_mapping), ("err", err)):
+        if t is not None:
+            _cuda(t, torch.int32, n)
+    _, ps, hkv, d = k_pool.shape
+    _check(lib.tv_pool_append_slots(
+        _ptr(state), num_pages, _ptr(block_tables), mb, _ptr(context_lens),
+        _ptr(num_new_tokens), b, _ptr(slot_mapping), _ptr(k_pool),
+        _ptr(v_pool), hkv, d, ps, _ptr(err), _stream(stream)),
+        "tv_pool_append_slots")
+
+
+def tv_pool_fork(state, block_tables, context_lens, src_seqs, dst_seqs,
+                 err=None, stream=None):
+    lib = load()
+    num_pages = _pool_pages(state)
+    mb, b = _pool_tables(block_tables, context_lens)
+    _cuda(src_seqs, torch.int32, "src_seqs"), _cuda(dst_seqs, torch.int32,
+                                                    "dst_seqs")
+    if src_seqs.shape != dst_seqs.shape:
+        raise ValueError("src_seqs and dst_seqs differ in length")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    _check(lib.tv_pool_fork(_ptr(state), num_pages, _ptr(block_tables), mb,
+                            _ptr(context_lens), b, _ptr(src_seqs),
+                            _ptr(dst_seqs), src_seqs.numel(), _ptr(err),
+                            _stream(stream)), "tv_pool_fork")
+
+
+def tv_pool_release(state, block_tables, context_lens, seqs, err=None,
+                    stream=None):
+    lib = load()
+    num_pages = _pool_pages(state)
+    mb, b = _pool_tables(block_tables, context_lens)
+    _cuda(seqs, torch.int32, "seqs")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    _check(lib.tv_pool_release(_ptr(state), num_pages, _ptr(block_tables), mb,
+                               _ptr(context_lens), b, _ptr(seqs), seqs.numel(),
+                               _ptr(err), _stream(stream)), "tv_pool_release")
+
+
+def tv_decode_step(state, out, q, k_new, v_new, k_pool, v_pool, block_tables,
+                   context_lens, scale, workspace=None, err=None, stream=None):
+    """Room for one new token per live sequence, then the fused append +
+    decode (two launches, no host synchronisation); with a workspace the
+    decode runs on the work-balanced grid."""
+    lib = load()
+    num_pages = _pool_pages(state)
+    mb, b = _pool_tables(block_tables, context_lens)
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_new", k_new), ("v_new", v_new),
+                 ("k_pool", k_pool), ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    if workspace is not None:
+        _cuda(workspace, torch.uint8, "workspace")
+    _, ps, hkv, d = k_pool.shape
+    hq = q.shape[1]
+    if out.shape != q.shape or q.shape[0] != b or k_new.shape != (b, hkv, d):
+        raise ValueError("shape mismatch")
+    _check(lib.tv_decode_step(
+        _ptr(state), num_pages, _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new),
+        _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), mb,
+        _ptr(context_lens), b, hq, hkv, d, ps, float(scale), _ptr(workspace),
+        workspace.numel() if workspace is not None else 0, _ptr(err),
+        _stream(stream)), "tv_decode_step")

@@ -346,6 +346,125 @@ tv_status tv_paged_decode_balanced(void* out, const void* q,
                        &ws);
 }
 
+// ---- device page pool ---------------------------------------------------------
+
+static tv_status pool_common(const int32_t* pool_state, int64_t num_pages,
+                             const int32_t* block_tables,
+                             int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs) {
+  if (!pool_state || num_pages <= 0 || num_seqs < 0 ||
+      (num_seqs > 0 &&
+       (!block_tables || !context_lens || max_blocks_per_seq <= 0)))
+    return TV_ERR_INVALID_ARG;
+  if (num_pages > (INT32_MAX - 4) / 4 || num_seqs > tv::kPoolMaxSeqs ||
+      (int64_t)max_blocks_per_seq * kPageSize > INT32_MAX)
+    return TV_ERR_UNSUPPORTED;
+  return TV_OK;
+}
+
+tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages,
+                       const int32_t* block_tables, int max_blocks_per_seq,
+                       const int32_t* context_lens, int num_seqs,
+                       uint32_t* err, void* stream) {
+  if (!block_tables) num_seqs = 0;
+  tv_status st = pool_common(pool_state, num_pages, block_tables,
+                             max_blocks_per_seq, context_lens, num_seqs);
+  if (st != TV_OK) return st;
+  return cuda_status(tv::launch_pool_init(
+      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      context_lens, num_seqs, err, static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_pool_append_slots(int32_t* pool_state, int64_t num_pages,
+                               int32_t* block_tables, int max_blocks_per_seq,
+                               int32_t* context_lens,
+                               const int32_t* num_new_tokens, int num_seqs,
+                               int32_t* slot_mapping, void* k_pool,
+                               void* v_pool, int num_kv_heads, int head_dim,
+                               int page_size, uint32_t* err, void* stream) {
+  tv_status st = pool_common(pool_state, num_pages, block_tables,
+                             max_blocks_per_seq, context_lens, num_seqs);
+  if (st != TV_OK) return st;
+  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (num_kv_heads <= 0 || !k_pool || !v_pool || !aligned16(k_pool) ||
+      !aligned16(v_pool))
+    return TV_ERR_INVALID_ARG;
+  if (num_seqs == 0) return TV_OK;
+  return cuda_status(tv::launch_pool_append(
+      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      context_lens, num_new_tokens, num_seqs, slot_mapping, k_pool, v_pool,
+      num_kv_heads * head_dim * 2, err, static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_pool_fork(int32_t* pool_state, int64_t num_pages,
+                       int32_t* block_tables, int max_blocks_per_seq,
+                       int32_t* context_lens, int num_seqs,
+                       const int32_t* src_seqs, const int32_t* dst_seqs,
+                       int num_pairs, uint32_t* err, void* stream) {
+  tv_status st = pool_common(pool_state, num_pages, block_tables,
+                             max_blocks_per_seq, context_lens, num_seqs);
+  if (st != TV_OK) return st;
+  if (num_pairs < 0 || (num_pairs > 0 && (!src_seqs || !dst_seqs)))
+    return TV_ERR_INVALID_ARG;
+  if (num_pairs == 0 || num_seqs == 0) return TV_OK;
+  return cuda_status(tv::launch_pool_fork(
+      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      context_lens, num_seqs, src_seqs, dst_seqs, num_pairs, err,
+      static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_pool_release(int32_t* pool_state, int64_t num_pages,
+                          int32_t* block_tables, int max_blocks_per_seq,
+                          int32_t* context_lens, int num_seqs,
+                          const int32_t* seqs, int num_release, uint32_t* err,
+                          void* stream) {
+  tv_status st = pool_common(pool_state, num_pages, block_tables,
+                             max_blocks_per_seq, context_lens, num_seqs);
+  if (st != TV_OK) return st;
+  if (num_release < 0 || (num_release > 0 && !seqs)) return TV_ERR_INVALID_ARG;
+  if (num_release == 0 || num_seqs == 0) return TV_OK;
+  return cuda_status(tv::launch_pool_release(
+      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      context_lens, num_seqs, seqs, num_release, err,
+      static_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_decode_step(int32_t* pool_state, int64_t num_pages, void* out,
+                         const void* q, const void* k_new, const void* v_new,
+                         void* k_pool, void* v_pool, int32_t* block_tables,
+                         int max_blocks_per_seq, int32_t* context_lens,
+                         int num_seqs, int num_q_heads, int num_kv_heads,
+                         int head_dim, int page_size, float scale,
+                         void* workspace, size_t workspace_bytes,
+                         uint32_t* err, void* stream) {
+  tv_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim,
+                                       page_size);
+  if (st != TV_OK) return st;
+  // check what the attention call checks before the pool is touched, so a
+  // rejected step changes nothing
+  if (!k_new || !v_new || !out || !q || !aligned16(out) || !aligned16(q) ||
+      !aligned16(k_new) || !aligned16(v_new) || !std::isfinite(scale) ||
+      num_pages * page_size > INT32_MAX ||
+      (workspace && !aligned16(workspace)))
+    return TV_ERR_INVALID_ARG;
+  st = tv_pool_append_slots(pool_state, num_pages, block_tables,
+                            max_blocks_per_seq, context_lens, nullptr,
+                            num_seqs, nullptr, k_pool, v_pool, num_kv_heads,
+                            head_dim, page_size, err, stream);
+  if (st != TV_OK) return st;
+  if (workspace)
+    return tv_paged_decode_balanced(
+        out, q, k_new, v_new, k_pool, v_pool, block_tables,
+        max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
+        head_dim, page_size, num_pages, scale, workspace, workspace_bytes, err,
+        stream);
+  return tv_paged_decode_append(out, q, k_new, v_new, k_pool, v_pool,
+                                block_tables, max_blocks_per_seq,
+                                context_lens, num_seqs, num_q_heads,
+                                num_kv_heads, head_dim, page_size, num_pages,
+                                scale, err, stream);
+}
+
 tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
                                 const void* q, const void* k_pool,
                                 const void* v_pool,

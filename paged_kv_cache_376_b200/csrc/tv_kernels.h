@@ -48,6 +48,29 @@ cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
                                 int num_seqs, int group, bool split,
                                 int parts, cudaStream_t stream);
 
+// Device page pool (page_pool.cu).  Error bits beyond those of tv_device.cuh.
+constexpr uint32_t DEVERR_POOL_EMPTY = 1u << 5;  // too few free pages
+constexpr uint32_t DEVERR_BAD_SEQ = 1u << 6;     // bad fork / release index
+constexpr int kPoolMaxSeqs = 1024;               // one thread per sequence
+
+cudaError_t launch_pool_init(int32_t* state, int num_pages,
+                             const int32_t* bt, int mb, const int32_t* ctx,
+                             int num_seqs, uint32_t* err, cudaStream_t stream);
+cudaError_t launch_pool_append(int32_t* state, int num_pages, int32_t* bt,
+                               int mb, int32_t* ctx, const int32_t* n_new,
+                               int num_seqs, int32_t* slot_mapping,
+                               void* k_pool, void* v_pool, int row_bytes,
+                               uint32_t* err, cudaStream_t stream);
+cudaError_t launch_pool_fork(int32_t* state, int num_pages, int32_t* bt,
+                             int mb, int32_t* ctx, int num_seqs,
+                             const int32_t* src, const int32_t* dst,
+                             int num_pairs, uint32_t* err,
+                             cudaStream_t stream);
+cudaError_t launch_pool_release(int32_t* state, int num_pages, int32_t* bt,
+                                int mb, int32_t* ctx, int num_seqs,
+                                const int32_t* seqs, int num_release,
+                                uint32_t* err, cudaStream_t stream);
+
 cudaError_t launch_kv_append(const void* k_new, const void* v_new,
                              const int32_t* slot_mapping, int64_t num_tokens,
                              void* k_pool, void* v_pool, int64_t num_slots,

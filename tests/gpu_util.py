@@ -34,6 +34,8 @@ def assert_parity(gpu, ref, what="", rel=REL, abs_=ABS):
     ref = np.asarray(ref, dtype=np.float64)
     assert g.shape == ref.shape, (g.shape, ref.shape)
     assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
+    # a NaN reference would make every comparison below vacuously true
+    assert np.isfinite(ref).all(), f"{what}: non-finite oracle output"
     err = np.abs(g - ref)
     bound = rel * np.abs(ref) + abs_
     bad = err > bound
