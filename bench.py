@@ -98,7 +98,7 @@ def _default_kind(name):
             "mix": "balanced"}.get(name, "fused")
 
 
-def _config(wl, name, kind=None):
+def _config(wl, name, kind=None, engine=False):
     kind = kind or _default_kind(name)
     cfg = {"workload": wl.name, "batch": wl.num_seqs,
            "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
@@ -121,6 +121,14 @@ def _config(wl, name, kind=None):
     else:
         cfg["step"] = "tv_kv_append (512-token chunks) + tv_paged_prefill"
         cfg["query_rows"] = int(wl.q.shape[0])
+    if engine:
+        cfg["step"] = ("tv_decode_step: device page pool slot reservation, "
+                       "then " + cfg["step"])
+        cfg["engine_state"] = (
+            "cache one token short of the workload; tables, lengths and "
+            f"pool state restored every {TVRunner.ENGINE_ROUND} steps by 3 "
+            "device copies inside the timed region, so contexts grow by up "
+            f"to {TVRunner.ENGINE_ROUND - 1} tokens within a round")
     kvb = wl.kv_bytes_read()
     cfg["l2"] = (f"inputs larger than L2: {kvb / 1e6:.0f} MB of K/V read per "
                  "step, streamed with an L2 evict-first policy"
@@ -189,8 +197,10 @@ class TVRunner:
     """Device buffers and the calls of one step, marshalled once so that the
     host submits a step in a few microseconds."""
 
+    ENGINE_ROUND = 64   # engine mode: steps between state restores
+
     def __init__(self, wl, name, device, unfused=False, split_tokens=0,
-                 per_pair=False, balanced=False):
+                 per_pair=False, balanced=False, engine=False):
         import torch
         from paged_kv_cache_376_b200 import _lib
         from paged_kv_cache_376_b200.device import upload
@@ -219,6 +229,45 @@ class TVRunner:
             self.maxp = maxp
         self.maxq = int(np.diff(wl.query_start_loc).max())
         self.stream = torch.cuda.current_stream(device)
+        self.engine = engine
+        if engine:
+            self._setup_engine()
+
+    def _setup_engine(self):
+        """Engine mode: the step is tv_decode_step on a device page pool.
+        The cache starts one token short of the workload (the step appends
+        it); the pools and tables get room for one round of growth, and the
+        tables, lengths and pool state are restored after every round so
+        each round repeats the same work."""
+        torch, db, wl = self.torch, self.db, self.wl
+        from paged_kv_cache_376_b200 import _lib
+        if self.kind not in ("fused", "balanced"):
+            raise SystemExit("--engine needs a decode workload")
+        b = wl.num_seqs
+        grow = self.ENGINE_ROUND // 16 + 2
+        shape = (b * grow,) + tuple(db.k_pool.shape[1:])
+        db.k_pool = torch.cat([db.k_pool, torch.zeros(
+            shape, dtype=db.k_pool.dtype, device=self.device)])
+        db.v_pool = torch.cat([db.v_pool, torch.zeros(
+            shape, dtype=db.v_pool.dtype, device=self.device)])
+        db.block_tables = torch.cat([db.block_tables, torch.full(
+            (b, grow), -1, dtype=torch.int32, device=self.device)], dim=1)
+        db.context_lens = (db.context_lens - 1).clamp_(min=0)
+        self.pool = _lib.pool_state(db.k_pool.shape[0], self.device)
+        _lib.tv_pool_init(self.pool, db.block_tables, db.context_lens)
+        self.saved = (db.block_tables.clone(), db.context_lens.clone(),
+                      self.pool.clone())
+        self.since_restore = 0
+        torch.cuda.synchronize(self.device)
+
+    def restore(self):
+        """Engine mode: back to the state at the start of a round."""
+        db = self.db
+        with self.torch.cuda.stream(self.stream):
+            db.block_tables.copy_(self.saved[0])
+            db.context_lens.copy_(self.saved[1])
+            self.pool.copy_(self.saved[2])
+        self.since_restore = 0
 
     def _p(self, t):
         import ctypes
@@ -232,6 +281,24 @@ class TVRunner:
         num_pages, ps, hkv, d = db.k_pool.shape
         b, hq = db.context_lens.shape[0], db.q.shape[1]
         mb = db.block_tables.shape[1]
+        if self.engine:
+            ws = self.ws if self.kind == "balanced" else None
+            if timing is not None:
+                timing[0].record(self.stream)
+            st = lib.tv_decode_step(
+                self._p(self.pool), num_pages, self._p(self.out),
+                self._p(db.q), self._p(db.k_new), self._p(db.v_new),
+                self._p(db.k_pool), self._p(db.v_pool),
+                self._p(db.block_tables), mb, self._p(db.context_lens), b, hq,
+                hkv, d, ps, wl.scale, self._p(ws) if ws is not None else None,
+                ws.numel() if ws is not None else 0, self._p(db.err), s)
+            assert st == 0, st
+            if timing is not None:
+                timing[1].record(self.stream)
+            self.since_restore += 1
+            if self.since_restore == self.ENGINE_ROUND:
+                self.restore()
+            return
         if self.kind == "balanced":
             if timing is not None:
                 timing[0].record(self.stream)
@@ -295,12 +362,24 @@ class TVRunner:
             assert st == 0, st
 
     def launches_per_step(self):
+        if self.engine:
+            return 2
         return {"split": 3, "fused": 1, "balanced": 1}.get(self.kind, 2)
+
+    def graph_timed(self):
+        """Steps timed by CUDA-graph replay: one launch per step, or the
+        engine's two launches with its restores."""
+        return self.engine or self.launches_per_step() == 1
 
     def graphs(self, steps, chunk=200):
         """CUDA graphs that replay exactly ``steps`` steps: a list of
-        graphs, each captured from ``chunk`` (or fewer) consecutive steps."""
+        graphs, each captured from ``chunk`` (or fewer) consecutive steps
+        (engine mode: rounds of ENGINE_ROUND steps, each ending with the
+        state restore)."""
         torch = self.torch
+        if self.engine:
+            chunk = self.ENGINE_ROUND
+            self.restore()
         cap = torch.cuda.Stream(self.device)
         cap.wait_stream(torch.cuda.current_stream(self.device))
         home, self.stream = self.stream, cap
@@ -320,6 +399,8 @@ class TVRunner:
         finally:
             self.stream = home
         torch.cuda.current_stream(self.device).wait_stream(cap)
+        if self.engine:
+            self.since_restore = 0
         return plan
 
     # -- end to end: host inputs in, host result out, through the C ABI ------
@@ -327,7 +408,13 @@ class TVRunner:
         torch = self.torch
         db = self.db
         self.h_in = {}
-        names = {"fused": ("q", "k_new", "v_new", "block_tables",
+        if self.engine:
+            # the engine's tables, lengths and pool stay on the device
+            self.restore()
+            names = ("q", "k_new", "v_new")
+        else:
+            names = None
+        names = names or {"fused": ("q", "k_new", "v_new", "block_tables",
                            "context_lens"),
                  "prefill": ("q", "k_new", "v_new", "slot_mapping",
                              "block_tables", "context_lens",
@@ -369,8 +456,8 @@ def run_tv(args, rank, world, local_rank):
     wl = _workload(args.workload)
     runner = TVRunner(wl, args.workload, device, unfused=args.unfused,
                       split_tokens=args.split_tokens, per_pair=args.per_pair,
-                      balanced=args.balanced)
-    use_graph = (runner.launches_per_step() == 1 and not args.eager)
+                      balanced=args.balanced, engine=args.engine)
+    use_graph = runner.graph_timed() and not args.eager
     per_step, unit, seqs = _units(wl, args.workload)
     hbm, tfl, tfl_sus, peak_src = _peaks()
     K, Wm = args.steps, args.warmup
@@ -440,6 +527,8 @@ def run_tv(args, rank, world, local_rank):
                    "tv_paged_decode_split", "prefill": "tv_paged_prefill",
                    "fused": "tv_paged_decode_append",
                    "balanced": "tv_paged_decode_balanced"}[runner.kind]
+    if runner.engine:
+        kernel_name = "tv_decode_step"
     if unit == "GB/s":
         peak, bound, src = hbm, "hbm", peak_src
     else:
@@ -452,7 +541,8 @@ def run_tv(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, shuffled "
         "page pool)",
-        "config": dict(_config(wl, args.workload, runner.kind),
+        "config": dict(_config(wl, args.workload, runner.kind,
+                               runner.engine),
                        parallelism=f"replicas{world}" if world > 1
                        else "single GPU",
                        launch=("CUDA graphs of up to 200 steps, replayed "
@@ -647,6 +737,9 @@ def main(argv=None):
     ap.add_argument("--balanced", action="store_true",
                     help="decode step as tv_paged_decode_balanced (the "
                          "work-balanced grid) with the append fused")
+    ap.add_argument("--engine", action="store_true",
+                    help="decode step as tv_decode_step on a device page "
+                         "pool (host-free, graph-captured engine step)")
     ap.add_argument("--eager", action="store_true",
                     help="launch every timed step from the host (no graph)")
     ap.add_argument("--split-tokens", type=int, default=0,
