@@ -86,11 +86,15 @@ def _traffic(kernel, workload_name):
         return None
 
 
-def _workload(name):
+def _workload(name, page_size=16):
     from paged_kv_cache_376_b200 import workloads as W
+    if name == "tiny":
+        if page_size != 16:
+            raise SystemExit("the tiny configuration has 16-token pages")
+        return W.tiny_decode()
     return {"llama": W.llama_decode, "mix": W.continuous_mix,
-            "long": W.long_split, "prefill": W.chunked_prefill,
-            "tiny": W.tiny_decode}[name]()
+            "long": W.long_split, "prefill": W.chunked_prefill}[name](
+                page_size=page_size)
 
 
 def _default_kind(name):
@@ -244,7 +248,7 @@ class TVRunner:
         if self.kind not in ("fused", "balanced"):
             raise SystemExit("--engine needs a decode workload")
         b = wl.num_seqs
-        grow = self.ENGINE_ROUND // 16 + 2
+        grow = self.ENGINE_ROUND // db.k_pool.shape[1] + 2
         shape = (b * grow,) + tuple(db.k_pool.shape[1:])
         db.k_pool = torch.cat([db.k_pool, torch.zeros(
             shape, dtype=db.k_pool.dtype, device=self.device)])
@@ -254,7 +258,8 @@ class TVRunner:
             (b, grow), -1, dtype=torch.int32, device=self.device)], dim=1)
         db.context_lens = (db.context_lens - 1).clamp_(min=0)
         self.pool = _lib.pool_state(db.k_pool.shape[0], self.device)
-        _lib.tv_pool_init(self.pool, db.block_tables, db.context_lens)
+        _lib.tv_pool_init(self.pool, db.block_tables, db.context_lens,
+                          page_size=db.k_pool.shape[1])
         self.saved = (db.block_tables.clone(), db.context_lens.clone(),
                       self.pool.clone())
         self.since_restore = 0
@@ -453,7 +458,7 @@ def run_tv(args, rank, world, local_rank):
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    wl = _workload(args.workload)
+    wl = _workload(args.workload, args.page_size)
     runner = TVRunner(wl, args.workload, device, unfused=args.unfused,
                       split_tokens=args.split_tokens, per_pair=args.per_pair,
                       balanced=args.balanced, engine=args.engine)
@@ -685,7 +690,7 @@ def cpu_baseline(wl, name, budget_s=12.0):
 
 def run_reference(args):
     import oracle
-    wl = _workload(args.workload)
+    wl = _workload(args.workload, args.page_size)
     cores = oracle.max_threads()
     K, Wm = args.steps, args.warmup
     # size the per-step sample so the whole run takes about two minutes
@@ -737,6 +742,9 @@ def main(argv=None):
     ap.add_argument("--balanced", action="store_true",
                     help="decode step as tv_paged_decode_balanced (the "
                          "work-balanced grid) with the append fused")
+    ap.add_argument("--page-size", type=int, default=16, choices=[16, 32],
+                    help="tokens per KV page (the workloads keep their "
+                         "contexts and pool bytes)")
     ap.add_argument("--engine", action="store_true",
                     help="decode step as tv_decode_step on a device page "
                          "pool (host-free, graph-captured engine step)")

@@ -26,13 +26,16 @@
  *       k_pool, v_pool   [num_pages][page_size][num_kv_heads][head_dim] bf16
  *                        (slot s = page s / page_size, offset s % page_size)
  *       block_tables     [num_seqs][max_blocks_per_seq] int32: physical page
- *                        of logical block b = token positions [16b, 16b+16)
+ *                        of logical block b = token positions
+ *                        [b*page_size, (b+1)*page_size)
  *       context_lens     [num_seqs] int32: tokens in the cache, counting the
  *                        ones just appended
  *       q, out (decode)  [num_seqs][num_q_heads][head_dim] bf16
  *       q, out (prefill) [total_query_rows][num_q_heads][head_dim] bf16
  *   - Query head h reads KV head h / (num_q_heads / num_kv_heads).
- *   - Supported: head_dim == 64, page_size == 16, num_q_heads a multiple of
+ *   - Supported: head_dim == 64, page_size 16 or 32 ([P3] recommends 16-32
+ *     tokens; the kernels stream 16-token blocks, two per 32-token page),
+ *     num_q_heads a multiple of
  *     num_kv_heads with a ratio in {1, 2, 4, 8}; every pointer 16-byte
  *     aligned.  Anything else returns TV_ERR_UNSUPPORTED or
  *     TV_ERR_INVALID_ARG before any launch.
@@ -136,7 +139,8 @@ tv_status tv_paged_decode(void* out, const void* q, const void* k_pool,
  * tv_paged_decode_append -- the whole decode step in one launch: append the
  * new token of every sequence at position context_lens[s]-1 (its slot found
  * through the block table) and attend over the cache, i.e. the result of
- * tv_kv_append with slot = block_tables[s][(ctx-1)/16]*16 + (ctx-1)%16
+ * tv_kv_append with slot = block_tables[s][(ctx-1)/PS]*PS + (ctx-1)%PS
+ * (PS = page_size)
  * followed by tv_paged_decode ([P1] "推理流程": compute the new token's K,V,
  * append them to the cache, then attend).  The new row is written to the
  * pools and used directly from shared memory, never read back from HBM.
@@ -322,7 +326,7 @@ tv_status tv_paged_decode_split_static(
  * caller-owned, set up by tv_pool_init and changed only by the tv_pool_*
  * calls:
  *   [0] number of free pages (top of the stack)   [2] slots written by the
- *   last tv_pool_append_slots   [4 .. 4+NP) free-page stack (pop takes entry
+ *   last tv_pool_append_slots   [3] page size   [4 .. 4+NP) free-page stack (pop takes entry
  *   top-1)   then NP reference counts and 2 x NP scratch words.
  * A page's reference count is the number of block-table rows holding it.
  * Every pool call serves at most 1024 sequences (TV_ERR_UNSUPPORTED above),
@@ -332,11 +336,14 @@ tv_status tv_paged_decode_split_static(
 
 /*
  * tv_pool_init -- every page free, except those the first
- * ceil(context_lens[s] / 16) entries of each block-table row hold (counted);
- * the free pages are stacked in descending id order, so a fresh pool hands
- * out pages 0, 1, 2, ...  block_tables may be NULL (an empty pool).
+ * ceil(context_lens[s] / page_size) entries of each block-table row hold
+ * (counted); the free pages are stacked in descending id order, so a fresh
+ * pool hands out pages 0, 1, 2, ...  block_tables may be NULL (an empty
+ * pool).  page_size (16 or 32) is kept in the state; every later pool call
+ * on it uses it (tv_pool_append_slots with another page_size flags
+ * TV_DEVERR_BAD_SEQ and changes nothing).
  */
-tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages,
+tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages, int page_size,
                        const int32_t* block_tables, int max_blocks_per_seq,
                        const int32_t* context_lens, int num_seqs,
                        uint32_t* err, void* stream);

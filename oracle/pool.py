@@ -43,19 +43,21 @@ import numpy as np
 PAGE = 16
 
 
-def pages_for(ctx: int) -> int:
-    return (int(ctx) + PAGE - 1) // PAGE
+def pages_for(ctx: int, page_size: int = PAGE) -> int:
+    return (int(ctx) + page_size - 1) // page_size
 
 
 class PagePool:
     """Free-page stack and reference counts of a pool of ``num_pages``."""
 
-    def __init__(self, num_pages: int, block_tables=None, context_lens=None):
+    def __init__(self, num_pages: int, block_tables=None, context_lens=None,
+                 page_size: int = PAGE):
         self.num_pages = int(num_pages)
+        self.ps = int(page_size)
         self.ref = np.zeros(self.num_pages, np.int64)
         if block_tables is not None:
             for s, ctx in enumerate(np.asarray(context_lens)):
-                for b in range(pages_for(ctx)):
+                for b in range(pages_for(ctx, self.ps)):
                     self.ref[int(block_tables[s][b])] += 1
         free = [p for p in range(self.num_pages) if self.ref[p] == 0]
         self.stack = list(reversed(free))     # top of stack = smallest id
@@ -72,6 +74,7 @@ class PagePool:
         """Make room for n_new[s] tokens per sequence (in place on the
         tables, lengths and pools).  Returns (slot_mapping, served mask)."""
         bt, ctx = block_tables, context_lens
+        ps = self.ps
         n_new = np.asarray(n_new, np.int64)
         # needs, reserved in batch order (all-or-nothing per sequence)
         ref_seen = self.ref.copy()     # counts as each sequence sees them
@@ -81,12 +84,12 @@ class PagePool:
             c, n = int(ctx[s]), int(n_new[s])
             if n <= 0:
                 continue
-            if c % PAGE:
-                p = int(bt[s][c // PAGE])
+            if c % ps:
+                p = int(bt[s][c // ps])
                 if ref_seen[p] > 1:
                     cow[s] = True
                     ref_seen[p] -= 1
-            need[s] = int(cow[s]) + pages_for(c + n) - pages_for(c)
+            need[s] = int(cow[s]) + pages_for(c + n, ps) - pages_for(c, ps)
         served = np.zeros(len(ctx), bool)
         used = 0
         for s in range(len(ctx)):
@@ -100,20 +103,20 @@ class PagePool:
             if n <= 0 or not served[s]:
                 continue
             if cow[s]:
-                old = int(bt[s][c // PAGE])
+                old = int(bt[s][c // ps])
                 new = self._pop()
                 self.ref[old] -= 1
                 self.ref[new] = 1
-                bt[s][c // PAGE] = new
+                bt[s][c // ps] = new
                 if k_pool is not None:
                     k_pool[new] = k_pool[old]
                     v_pool[new] = v_pool[old]
-            for b in range(pages_for(c), pages_for(c + n)):
+            for b in range(pages_for(c, ps), pages_for(c + n, ps)):
                 new = self._pop()
                 self.ref[new] = 1
                 bt[s][b] = new
             for t in range(c, c + n):
-                slots.append(int(bt[s][t // PAGE]) * PAGE + t % PAGE)
+                slots.append(int(bt[s][t // ps]) * ps + t % ps)
             ctx[s] = c + n
         return np.array(slots, np.int32), served
 
@@ -121,7 +124,7 @@ class PagePool:
         """Drop every page reference of the sequences ``seqs``."""
         freed = set()
         for s in seqs:
-            for b in range(pages_for(context_lens[s])):
+            for b in range(pages_for(context_lens[s], self.ps)):
                 p = int(block_tables[s][b])
                 self.ref[p] -= 1
                 if self.ref[p] == 0:
@@ -134,7 +137,7 @@ class PagePool:
     def fork(self, block_tables, context_lens, pairs):
         """For every (src, dst): dst (empty) shares src's pages."""
         for src, dst in pairs:
-            n = pages_for(context_lens[src])
+            n = pages_for(context_lens[src], self.ps)
             block_tables[dst][:] = -1
             block_tables[dst][:n] = block_tables[src][:n]
             for b in range(n):

@@ -54,7 +54,7 @@ SIGNATURES = {
     "tv_paged_decode_balanced": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
                                       _I, _I, _I, _I, _I64, _F, _P,
                                       ctypes.c_size_t, _P, _P]),
-    "tv_pool_init": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P]),
+    "tv_pool_init": (_I, [_P, _I64, _I, _P, _I, _P, _I, _P, _P]),
     "tv_pool_append_slots": (_I, [_P, _I64, _P, _I, _P, _P, _I, _P, _P, _P,
                                   _I, _I, _I, _P, _P]),
     "tv_pool_fork": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P, _I, _P, _P]),
@@ -378,14 +378,15 @@ def _pool_pages(state):
 
 
 def tv_pool_init(state, block_tables=None, context_lens=None, err=None,
-                 stream=None):
+                 stream=None, page_size=16):
     lib = load()
     num_pages = _pool_pages(state)
     mb, b = (_pool_tables(block_tables, context_lens)
              if block_tables is not None else (0, 0))
     if err is not None:
         _cuda(err, torch.int32, "err")
-    _check(lib.tv_pool_init(_ptr(state), num_pages, _ptr(block_tables), mb,
+    _check(lib.tv_pool_init(_ptr(state), num_pages, int(page_size),
+                            _ptr(block_tables), mb,
                             _ptr(context_lens), b, _ptr(err),
                             _stream(stream)), "tv_pool_init")
 

@@ -33,12 +33,12 @@
 namespace tv {
 namespace {
 
-constexpr int kPS = 16;
 constexpr int kThreads = 1024;
 
 struct PoolView {
   int32_t* top;
   int32_t* last_slots;   // slots written by the last append call
+  int32_t* page_size;    // tokens per page, set by init (16 or 32)
   int32_t* stack;        // [num_pages]
   int32_t* ref;          // [num_pages]
   int32_t* cnt_app;      // [num_pages], zero between calls
@@ -50,6 +50,7 @@ __host__ __device__ inline PoolView view(int32_t* state, int num_pages) {
   PoolView v;
   v.top = state + 0;
   v.last_slots = state + 2;
+  v.page_size = state + 3;
   v.stack = state + 4;
   v.ref = v.stack + num_pages;
   v.cnt_app = v.ref + num_pages;
@@ -58,8 +59,8 @@ __host__ __device__ inline PoolView view(int32_t* state, int num_pages) {
   return v;
 }
 
-__device__ __forceinline__ int pages_for(int ctx) {
-  return (ctx + kPS - 1) / kPS;
+__device__ __forceinline__ int pages_for(int ctx, int ps) {
+  return (ctx + ps - 1) / ps;
 }
 
 // Exclusive scan of one int per thread over the 1024 threads of the CTA;
@@ -104,7 +105,7 @@ __global__ void pool_clear_kernel(PoolView p) {
 
 __global__ void pool_count_refs_kernel(PoolView p, const int32_t* bt, int mb,
                                        const int32_t* ctx, int num_seqs,
-                                       uint32_t* err) {
+                                       int kPS, uint32_t* err) {
   const int64_t total = (int64_t)num_seqs * mb;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -114,7 +115,7 @@ __global__ void pool_count_refs_kernel(PoolView p, const int32_t* bt, int mb,
       if (b == 0) flag_error(err, DEVERR_BAD_CONTEXT);
       c = c < 0 ? 0 : mb * kPS;
     }
-    if (b >= pages_for(c)) continue;
+    if (b >= pages_for(c, kPS)) continue;
     const int page = bt[(size_t)s * mb + b];
     if (page < 0 || page >= p.num_pages) {
       flag_error(err, DEVERR_BAD_PAGE);
@@ -125,7 +126,8 @@ __global__ void pool_count_refs_kernel(PoolView p, const int32_t* bt, int mb,
 }
 
 // stack = unreferenced pages in descending id order (a fresh pool pops 0, 1..)
-__global__ void __launch_bounds__(kThreads, 1) pool_stack_kernel(PoolView p) {
+__global__ void __launch_bounds__(kThreads, 1)
+    pool_stack_kernel(PoolView p, int page_size) {
   __shared__ int sh[33];
   int base = 0;
   for (int i0 = 0; i0 < p.num_pages; i0 += kThreads) {
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) pool_stack_kernel(PoolView p) {
   if (threadIdx.x == 0) {
     *p.top = base;
     *p.last_slots = 0;
+    *p.page_size = page_size;
   }
 }
 
@@ -149,9 +152,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     pool_append_kernel(PoolView p, int32_t* bt, int mb, int32_t* ctx,
                        const int32_t* n_new, int num_seqs,
                        int32_t* slot_mapping, uint8_t* k_pool,
-                       uint8_t* v_pool, int row_bytes, uint32_t* err) {
+                       uint8_t* v_pool, int row_bytes, int kPS,
+                       uint32_t* err) {
   __shared__ int sh[33];
   __shared__ int job_old[kThreads], job_new[kThreads];
+  if (*p.page_size != kPS) {   // pools of another page size: touch nothing
+    if (threadIdx.x == 0) flag_error(err, DEVERR_BAD_SEQ);
+    return;
+  }
   const int s = threadIdx.x;
   const bool live = s < num_seqs;
   int c = 0, n = 0, part = -1;
@@ -183,7 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = p.ref[part];
     cow = r > 1 && !(p.cnt_app[part] == r && p.last_app[part] == s + 1);
   }
-  const int need = n > 0 ? (int)cow + pages_for(c + n) - pages_for(c) : 0;
+  const int need =
+      n > 0 ? (int)cow + pages_for(c + n, kPS) - pages_for(c, kPS) : 0;
   const int top = *p.top;
   int total;
   const int off = block_exclusive_scan(need, sh, &total);
@@ -208,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       job_new[s] = fresh;
       job = s;
     }
-    for (int b = pages_for(c); b < pages_for(c + n); ++b) {
+    for (int b = pages_for(c, kPS); b < pages_for(c + n, kPS); ++b) {
       const int fresh = p.stack[k--];
       bt[(size_t)s * mb + b] = fresh;
       p.ref[fresh] = 1;
@@ -256,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pool_fork_kernel(PoolView p, int32_t* bt, int mb, int32_t* ctx,
                      int num_seqs, const int32_t* src, const int32_t* dst,
                      int num_pairs, uint32_t* err) {
+  const int kPS = *p.page_size;
   for (int i = 0; i < num_pairs; ++i) {
     const int a = src[i], b = dst[i];
     bool ok = a >= 0 && a < num_seqs && b >= 0 && b < num_seqs && a != b;
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       continue;
     }
-    const int np = pages_for(c);
+    const int np = pages_for(c, kPS);
     for (int k = threadIdx.x; k < mb; k += kThreads) {
       const int page = k < np ? bt[(size_t)a * mb + k] : -1;
       bt[(size_t)b * mb + k] = page;
@@ -287,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int sh[33];
   __shared__ int freed[kList];
   __shared__ int nfreed;
+  const int kPS = *p.page_size;
   if (threadIdx.x == 0) nfreed = 0;
   __syncthreads();
   for (int i = 0; i < num_release; ++i) {
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int c = ctx[s];
     c = c < 0 ? 0 : (c > mb * kPS ? mb * kPS : c);
-    const int np = pages_for(c);
+    const int np = pages_for(c, kPS);
     for (int k = threadIdx.x; k < mb; k += kThreads) {
       if (k < np) {
         const int page = bt[(size_t)s * mb + k];
@@ -365,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_pool_init(int32_t* state, int num_pages,
+cudaError_t launch_pool_init(int32_t* state, int num_pages, int page_size,
                              const int32_t* bt, int mb, const int32_t* ctx,
                              int num_seqs, uint32_t* err,
                              cudaStream_t stream) {
@@ -375,21 +386,22 @@ cudaError_t launch_pool_init(int32_t* state, int num_pages,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   pool_clear_kernel<<<sms, 256, 0, stream>>>(p);
   if (bt && num_seqs > 0)
-    pool_count_refs_kernel<<<sms * 4, 256, 0, stream>>>(p, bt, mb, ctx,
-                                                        num_seqs, err);
-  pool_stack_kernel<<<1, kThreads, 0, stream>>>(p);
+    pool_count_refs_kernel<<<sms * 4, 256, 0, stream>>>(
+        p, bt, mb, ctx, num_seqs, page_size, err);
+  pool_stack_kernel<<<1, kThreads, 0, stream>>>(p, page_size);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool_append(int32_t* state, int num_pages, int32_t* bt,
-                               int mb, int32_t* ctx, const int32_t* n_new,
-                               int num_seqs, int32_t* slot_mapping,
-                               void* k_pool, void* v_pool, int row_bytes,
-                               uint32_t* err, cudaStream_t stream) {
+cudaError_t launch_pool_append(int32_t* state, int num_pages, int page_size,
+                               int32_t* bt, int mb, int32_t* ctx,
+                               const int32_t* n_new, int num_seqs,
+                               int32_t* slot_mapping, void* k_pool,
+                               void* v_pool, int row_bytes, uint32_t* err,
+                               cudaStream_t stream) {
   pool_append_kernel<<<1, kThreads, 0, stream>>>(
       view(state, num_pages), bt, mb, ctx, n_new, num_seqs, slot_mapping,
       static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool),
-      row_bytes, err);
+      row_bytes, page_size, err);
   return cudaGetLastError();
 }
 

@@ -82,7 +82,11 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
   // ---- token range of this CTA --------------------------------------------
   int ctx = a.context_lens[seq];
-  const int ctx_cap = a.max_blocks_per_seq * kPS;
+  // A page holds 1 << page_shift blocks of 16 tokens; the kernel streams
+  // blocks, and a block's 16 rows are one TMA box at row (page << shift |
+  // sub-block) * 16 of the pool.
+  const int ctx_cap = a.max_blocks_per_seq * (kPS << a.page_shift);
+  const int num_blocks = a.num_pages << a.page_shift;
   if (ctx < 0 || ctx > ctx_cap) {
     if (threadIdx.x == 0) flag_error(a.err, DEVERR_BAD_CONTEXT);
     ctx = ctx < 0 ? 0 : ctx_cap;
@@ -97,8 +101,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int n_pages = (tok_end - tok_begin + kPS - 1) / kPS;
   // pages of this warp: first_page + warp + kWarps * i, i < my_n
   const int my_n = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
-  const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq +
-                      first_page + warp;
+  const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
+  const int sub_mask = (1 << a.page_shift) - 1;
 
   // ---- fused append: the new token is at position ctx-1 (unsplit kernel) ---
   int app_i = -1;            // local page index of the appended row, this warp
@@ -156,17 +160,22 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc2[h][i] = make_float2(0.f, 0.f);
 
-  // Block-table entries of this warp's pages, 32 per batch, one per lane.
+  // Pool blocks of this warp's 16-token blocks, 32 per batch, one per lane
+  // (-1 when the block-table entry is not a page of the pool).
   auto load_pids = [&](int batch) -> int {
     const int i = batch * 32 + lane;
-    return i < my_n ? __ldg(bt + (size_t)i * kWarps) : 0;
+    if (i >= my_n) return 0;
+    const int b = first_page + warp + kWarps * i;
+    const int page = __ldg(bt + (b >> a.page_shift));
+    return page >= 0 && page < a.num_pages
+               ? (page << a.page_shift) + (b & sub_mask) : -1;
   };
   int pid_cur = load_pids(0);
   int pid_next = load_pids(1);
   const uint64_t policy = l2_policy_evict_first();
 
   auto issue = [&](int pid, int stage) {
-    const bool ok = pid >= 0 && pid < a.num_pages;
+    const bool ok = pid >= 0 && pid < num_blocks;
     if (!ok) flag_error(a.err, DEVERR_BAD_PAGE);
     const int y = (ok ? pid : 0) * kPS;
     const uint32_t bar = smem_u32(&sm.full[warp][stage]);
@@ -194,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       pid_next = load_pids((i >> 5) + 1);
     }
     const int pid = __shfl_sync(0xffffffffu, pid_cur, i & 31);
-    const bool page_ok = pid >= 0 && pid < a.num_pages;
+    const bool page_ok = pid >= 0 && pid < num_blocks;
     const int page_tok0 = (first_page + warp + kWarps * i) * kPS;
     // warp-uniform: every token of the page is a real key of this range
     const bool full_page = page_ok && page_tok0 + kPS <= tok_end;

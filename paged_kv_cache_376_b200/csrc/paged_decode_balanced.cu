@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int chk = lane & 7;
   const int B = a.num_seqs;
   const int Hkv = a.num_kv_heads;
-  const int ctx_cap = a.max_blocks_per_seq * kPS;
+  // a page holds 1 << page_shift blocks of 16 tokens; the work unit here is
+  // the 16-token block (one TMA box)
+  const int ctx_cap = a.max_blocks_per_seq * (kPS << a.page_shift);
 
   // ---- pages per sequence, exclusive prefix in shared memory ---------------
   for (int s = threadIdx.x; s < B; s += kThreads) {
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   };
 
   // ---- per-lane page table: positions x0 + 32*batch + lane -----------------
-  // One word per page: bits 0-25 the physical page (kNoPage when nothing is
+  // One word per 16-token block: bits 0-25 the pool block (kNoPage when nothing is
   // to be loaded: empty context or a bad block-table entry), bit 26 first
   // page of its sequence, bit 27 last page, bits 28-31 valid tokens - 1
   // (15 on every page but the last).  seq0 receives the sequence of the
@@ -204,12 +206,14 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
       const int p = x - sm.pre[lo];
       const bool last = x == sm.pre[lo + 1] - 1;
       const int lv = sm.last_valid[lo];
-      uint32_t pid = kNoPage;
+      uint32_t pid = kNoPage;   // the pool block (16 rows) of this block
       if (lv > 0) {
-        const int raw =
-            __ldg(a.block_tables + (size_t)lo * a.max_blocks_per_seq + p);
+        const int raw = __ldg(a.block_tables +
+                              (size_t)lo * a.max_blocks_per_seq +
+                              (p >> a.page_shift));
         if (raw >= 0 && raw < a.num_pages) {
-          pid = (uint32_t)raw;
+          pid = ((uint32_t)raw << a.page_shift) +
+                (uint32_t)(p & ((1 << a.page_shift) - 1));
         } else if (head == 0) {
           flag_error(a.err, DEVERR_BAD_PAGE);
         }

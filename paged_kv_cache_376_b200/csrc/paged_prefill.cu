@@ -104,7 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qs = a.query_start_loc[seq];
   const int T = a.query_start_loc[seq + 1] - qs;
   int ctx = a.context_lens[seq];
-  const int ctx_cap = a.max_blocks_per_seq * kPS;
+  // a page holds 1 << page_shift blocks of 16 tokens, each one TMA box
+  const int ctx_cap = a.max_blocks_per_seq * (kPS << a.page_shift);
   const int q0 = blk * kQRows * kQTiles;
   if (q0 >= T) return;
   if (ctx > ctx_cap) {
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kQTiles; ++t)
         tma_load_3d(smem_u32(sm.q[t]), &tm_q, 0, kvh * kG,
                     qs + q0 + t * kQRows, qbar);
-      const int oob_row = a.num_pages * kPS;   // reads as zeros
+      const int oob_row = (a.num_pages << a.page_shift) * kPS;  // zeros
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j % kST;
         if (j >= kST &&
@@ -178,9 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int lp = j * kPagesPerTile + p;
           int y = oob_row;
           if (lp < n_pages) {
-            const int pid = __ldg(bt + lp);
+            const int pid = __ldg(bt + (lp >> a.page_shift));
             if (pid >= 0 && pid < a.num_pages) {
-              y = pid * kPS;
+              y = ((pid << a.page_shift) + (lp & ((1 << a.page_shift) - 1))) *
+                  kPS;
             } else {
               bad |= 1u << p;
             }

@@ -19,7 +19,12 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kHeadDim = 64;
-constexpr int kPageSize = 16;
+constexpr int kPageSize = 16;   // the kernels' block: 16 token rows
+
+// Pages of 16 or 32 tokens ([P3] 内存池管理 recommends 16-32); a page is
+// 1 << page_shift blocks of 16 rows.
+bool page_size_ok(int page_size) { return page_size == 16 || page_size == 32; }
+int page_shift(int page_size) { return page_size == 32 ? 1 : 0; }
 
 tv_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return TV_OK;
@@ -55,17 +60,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // The pool seen as a 2-D bf16 tensor [num_pages * page_size][Hkv * D]; the
-// box is one page of one KV head: 16 rows x 64 elements (128 B).  The 256-byte
+// box is one 16-token block of one KV head: 16 rows x 64 elements (128 B)
+// (a 32-token page is two boxes).  The 256-byte
 // L2 promotion also fetches the neighbouring KV head's row; every decode grid
 // reads the KV heads of a page at about the same time, so that row is an L2
 // hit for its reader, not a second DRAM read.
 tv_status pool_tensor_map(CUtensorMap* map, const void* pool,
-                          int64_t num_pages, int num_kv_heads,
+                          int64_t num_pages, int page_size, int num_kv_heads,
                           CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return TV_ERR_CUDA;
   const cuuint64_t dims[2] = {(cuuint64_t)num_kv_heads * kHeadDim,
-                              (cuuint64_t)num_pages * kPageSize};
+                              (cuuint64_t)num_pages * page_size};
   const cuuint64_t strides[1] = {(cuuint64_t)num_kv_heads * kHeadDim * 2};
   const cuuint32_t box[2] = {kHeadDim, kPageSize};
   const cuuint32_t estr[2] = {1, 1};
@@ -109,7 +115,8 @@ tv_status query_tensor_map(CUtensorMap* map, const void* q, int64_t rows,
 
 tv_status check_attention_shape(int num_q_heads, int num_kv_heads,
                                 int head_dim, int page_size) {
-  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (head_dim != kHeadDim || !page_size_ok(page_size))
+    return TV_ERR_UNSUPPORTED;
   if (!group_ok(num_q_heads, num_kv_heads)) return TV_ERR_UNSUPPORTED;
   return TV_OK;
 }
@@ -140,7 +147,8 @@ tv_status tv_kv_append(const void* k_new, const void* v_new,
                        uint32_t* err, void* stream) {
   if (num_tokens < 0 || num_pages <= 0 || num_kv_heads <= 0)
     return TV_ERR_INVALID_ARG;
-  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (head_dim != kHeadDim || !page_size_ok(page_size))
+    return TV_ERR_UNSUPPORTED;
   if (num_tokens == 0) return TV_OK;
   if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
     return TV_ERR_INVALID_ARG;
@@ -221,16 +229,17 @@ static tv_status decode_common(void* out, float* partial_out,
   if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
     return TV_ERR_INVALID_ARG;
 
+  const int shift = page_shift(page_size);
   const bool balanced = ws && num_seqs <= tv::kMaxBalancedSeqs &&
                         max_blocks_per_seq < (1 << 24) &&
-                        num_pages < (1 << 26) - 1 &&
+                        (num_pages << shift) < (1 << 26) - 1 &&
                         (int64_t)num_seqs * num_kv_heads *
-                                max_blocks_per_seq < INT32_MAX;
+                                (max_blocks_per_seq << shift) < INT32_MAX;
   CUtensorMap tk, tvm;
-  st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
+  st = pool_tensor_map(&tk, k_pool, num_pages, page_size, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != TV_OK) return st;
-  st = pool_tensor_map(&tvm, v_pool, num_pages, num_kv_heads,
+  st = pool_tensor_map(&tvm, v_pool, num_pages, page_size, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != TV_OK) return st;
 
@@ -252,6 +261,7 @@ static tv_status decode_common(void* out, float* partial_out,
   a.partition_tokens = split ? partition_tokens : 0;
   a.max_partitions = split ? max_partitions : 1;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.page_shift = shift;
   const int group = num_q_heads / num_kv_heads;
   // The balanced grid needs the prefix sums of every sequence in shared
   // memory, all flattened page positions in int32, page indices in 24 bits
@@ -265,8 +275,9 @@ static tv_status decode_common(void* out, float* partial_out,
     if (ws->bytes < cb + partials_bytes(cap)) return TV_ERR_INVALID_ARG;
     // groups of num_kv_heads warps, each with >= kMinPagesPerWarp pages
     // (num_seqs * max_blocks_per_seq bounds the page count from above)
-    const int64_t groups = ((int64_t)num_seqs * max_blocks_per_seq +
-                            tv::kMinPagesPerWarp - 1) / tv::kMinPagesPerWarp;
+    const int64_t groups =
+        ((int64_t)num_seqs * (max_blocks_per_seq << shift) +
+         tv::kMinPagesPerWarp - 1) / tv::kMinPagesPerWarp;
     const int64_t want = (groups * num_kv_heads + 3) / 4;
     const int64_t least = (num_kv_heads + 3) / 4;   // one whole group
     if (cap < least) return TV_ERR_UNSUPPORTED;
@@ -357,12 +368,12 @@ static tv_status pool_common(const int32_t* pool_state, int64_t num_pages,
        (!block_tables || !context_lens || max_blocks_per_seq <= 0)))
     return TV_ERR_INVALID_ARG;
   if (num_pages > (INT32_MAX - 4) / 4 || num_seqs > tv::kPoolMaxSeqs ||
-      (int64_t)max_blocks_per_seq * kPageSize > INT32_MAX)
+      (int64_t)max_blocks_per_seq * 32 > INT32_MAX)
     return TV_ERR_UNSUPPORTED;
   return TV_OK;
 }
 
-tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages,
+tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages, int page_size,
                        const int32_t* block_tables, int max_blocks_per_seq,
                        const int32_t* context_lens, int num_seqs,
                        uint32_t* err, void* stream) {
@@ -370,8 +381,9 @@ tv_status tv_pool_init(int32_t* pool_state, int64_t num_pages,
   tv_status st = pool_common(pool_state, num_pages, block_tables,
                              max_blocks_per_seq, context_lens, num_seqs);
   if (st != TV_OK) return st;
+  if (!page_size_ok(page_size)) return TV_ERR_UNSUPPORTED;
   return cuda_status(tv::launch_pool_init(
-      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      pool_state, (int)num_pages, page_size, block_tables, max_blocks_per_seq,
       context_lens, num_seqs, err, static_cast<cudaStream_t>(stream)));
 }
 
@@ -385,13 +397,14 @@ tv_status tv_pool_append_slots(int32_t* pool_state, int64_t num_pages,
   tv_status st = pool_common(pool_state, num_pages, block_tables,
                              max_blocks_per_seq, context_lens, num_seqs);
   if (st != TV_OK) return st;
-  if (head_dim != kHeadDim || page_size != kPageSize) return TV_ERR_UNSUPPORTED;
+  if (head_dim != kHeadDim || !page_size_ok(page_size))
+    return TV_ERR_UNSUPPORTED;
   if (num_kv_heads <= 0 || !k_pool || !v_pool || !aligned16(k_pool) ||
       !aligned16(v_pool))
     return TV_ERR_INVALID_ARG;
   if (num_seqs == 0) return TV_OK;
   return cuda_status(tv::launch_pool_append(
-      pool_state, (int)num_pages, block_tables, max_blocks_per_seq,
+      pool_state, (int)num_pages, page_size, block_tables, max_blocks_per_seq,
       context_lens, num_new_tokens, num_seqs, slot_mapping, k_pool, v_pool,
       num_kv_heads * head_dim * 2, err, static_cast<cudaStream_t>(stream)));
 }
@@ -536,10 +549,10 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   st = query_tensor_map(&tq, q, num_query_rows, num_q_heads,
                         num_q_heads / num_kv_heads, 32);
   if (st != TV_OK) return st;
-  st = pool_tensor_map(&tk, k_pool, num_pages, num_kv_heads,
+  st = pool_tensor_map(&tk, k_pool, num_pages, page_size, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != TV_OK) return st;
-  st = pool_tensor_map(&tvm, v_pool, num_pages, num_kv_heads,
+  st = pool_tensor_map(&tvm, v_pool, num_pages, page_size, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != TV_OK) return st;
 
@@ -557,6 +570,7 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   a.max_query_len = max_query_len;
   a.num_query_rows = num_query_rows;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.page_shift = page_shift(page_size);
   return cuda_status(tv::launch_paged_prefill(
       a, tq, tk, tvm, static_cast<cudaStream_t>(stream)));
 }

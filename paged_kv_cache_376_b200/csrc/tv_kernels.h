@@ -26,6 +26,7 @@ struct DecodeArgs {
   int partition_tokens;
   int max_partitions;
   float scale_log2;              // scale * log2(e)
+  int page_shift;                // page_size = 16 << page_shift
   // work-balanced decode only
   int num_seqs;
   int num_kv_heads;
@@ -53,14 +54,15 @@ constexpr uint32_t DEVERR_POOL_EMPTY = 1u << 5;  // too few free pages
 constexpr uint32_t DEVERR_BAD_SEQ = 1u << 6;     // bad fork / release index
 constexpr int kPoolMaxSeqs = 1024;               // one thread per sequence
 
-cudaError_t launch_pool_init(int32_t* state, int num_pages,
+cudaError_t launch_pool_init(int32_t* state, int num_pages, int page_size,
                              const int32_t* bt, int mb, const int32_t* ctx,
                              int num_seqs, uint32_t* err, cudaStream_t stream);
-cudaError_t launch_pool_append(int32_t* state, int num_pages, int32_t* bt,
-                               int mb, int32_t* ctx, const int32_t* n_new,
-                               int num_seqs, int32_t* slot_mapping,
-                               void* k_pool, void* v_pool, int row_bytes,
-                               uint32_t* err, cudaStream_t stream);
+cudaError_t launch_pool_append(int32_t* state, int num_pages, int page_size,
+                               int32_t* bt, int mb, int32_t* ctx,
+                               const int32_t* n_new, int num_seqs,
+                               int32_t* slot_mapping, void* k_pool,
+                               void* v_pool, int row_bytes, uint32_t* err,
+                               cudaStream_t stream);
 cudaError_t launch_pool_fork(int32_t* state, int num_pages, int32_t* bt,
                              int mb, int32_t* ctx, int num_seqs,
                              const int32_t* src, const int32_t* dst,
@@ -97,6 +99,7 @@ struct PrefillArgs {
   int max_query_len;
   int64_t num_query_rows;
   float scale_log2;
+  int page_shift;                // page_size = 16 << page_shift
 };
 
 cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,

@@ -267,16 +267,23 @@ def tiny_decode() -> Workload:
                            seed=SEED_BASE + 1, name="tiny-decode")
 
 
+def _ps_tag(page_size: int) -> str:
+    return "" if page_size == PAGE_SIZE else f"-ps{page_size}"
+
+
 def llama_decode(batch: int = 64, context: int = 2048,
-                 num_pages: int = 16384) -> Workload:
-    """Llama-3.2-1B-shaped decode: 64 sequences x 2048 tokens, 16384-page
-    shuffled pool (half used)."""
+                 num_pages: int = 16384, page_size: int = PAGE_SIZE
+                 ) -> Workload:
+    """Llama-3.2-1B-shaped decode: 64 sequences x 2048 tokens, a shuffled
+    pool twice the size of the cache (16384 pages of 16 tokens)."""
+    num_pages = num_pages * PAGE_SIZE // page_size
     return decode_workload([context] * batch, num_pages=num_pages,
-                           seed=SEED_BASE + 2,
-                           name=f"llama3.2-1b-decode-b{batch}-ctx{context}")
+                           seed=SEED_BASE + 2, page_size=page_size,
+                           name=f"llama3.2-1b-decode-b{batch}-ctx{context}"
+                                + _ps_tag(page_size))
 
 
-def continuous_mix(batch: int = 256) -> Workload:
+def continuous_mix(batch: int = 256, page_size: int = PAGE_SIZE) -> Workload:
     """Continuous-batching mix: contexts log-uniform in [16, 8192]; a context
     whose appended token would open a new page is bumped by one, so every
     append lands in a partly filled last page."""
@@ -285,33 +292,38 @@ def continuous_mix(batch: int = 256) -> Workload:
     ctx = np.rint(np.exp(rng.uniform(math.log(16), math.log(8192),
                                      size=batch))).astype(np.int64)
     ctx = np.where((ctx - 1) % PAGE_SIZE == 0, ctx + 1, ctx)
-    num_pages = int(sum(-(-int(n) // PAGE_SIZE) for n in ctx))
-    return _build(f"continuous-mix-b{batch}", seed, ctx - 1,
-                  np.ones_like(ctx), num_pages, kind="decode", rng=rng)
+    num_pages = int(sum(-(-int(n) // page_size) for n in ctx))
+    return _build(f"continuous-mix-b{batch}" + _ps_tag(page_size), seed,
+                  ctx - 1, np.ones_like(ctx), num_pages, kind="decode",
+                  rng=rng, page_size=page_size)
 
 
 def long_split(batch: int = 8, context: int = 131072,
-               partition_tokens: int = 512) -> Workload:
+               partition_tokens: int = 512, page_size: int = PAGE_SIZE
+               ) -> Workload:
     """Long-context split-KV decode: 8 x 131072 tokens, 512-token
     partitions merged by log-sum-exp."""
-    num_pages = batch * context // PAGE_SIZE
+    num_pages = batch * context // page_size
     return decode_workload([context] * batch, num_pages=num_pages,
-                           seed=SEED_BASE + 4,
-                           name=f"long-split-b{batch}-ctx{context}",
+                           seed=SEED_BASE + 4, page_size=page_size,
+                           name=f"long-split-b{batch}-ctx{context}"
+                                + _ps_tag(page_size),
                            partition_tokens=partition_tokens)
 
 
 def chunked_prefill(batch: int = 16, chunk: int = 512,
-                    max_prefix: int = 4096) -> Workload:
+                    max_prefix: int = 4096, page_size: int = PAGE_SIZE
+                    ) -> Workload:
     """Chunked prefill: 16 sequences, 512 new tokens each over a cached
     prefix drawn uniformly from {0 .. 4096}."""
     seed = SEED_BASE + 5
     rng = np.random.Generator(np.random.PCG64(seed))
     pre = rng.integers(0, max_prefix + 1, size=batch).astype(np.int64)
     chunks = np.full((batch,), chunk, dtype=np.int64)
-    num_pages = int(sum(-(-int(n) // PAGE_SIZE) for n in pre + chunks))
-    return _build(f"chunked-prefill-b{batch}-chunk{chunk}", seed, pre,
-                  chunks, num_pages, kind="prefill", rng=rng)
+    num_pages = int(sum(-(-int(n) // page_size) for n in pre + chunks))
+    return _build(f"chunked-prefill-b{batch}-chunk{chunk}"
+                  + _ps_tag(page_size), seed, pre, chunks, num_pages,
+                  kind="prefill", rng=rng, page_size=page_size)
 
 
 NAMED = {

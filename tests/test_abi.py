@@ -52,9 +52,10 @@ def test_unsupported_shapes_are_rejected_before_launch(lib):
     # head_dim 128
     assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 128, 16, 10,
                                0.1, None, None) == 2
-    # page size 32
-    assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 64, 32, 10,
-                               0.1, None, None) == 2
+    # page sizes other than 16 and 32
+    for ps in (8, 24, 64):
+        assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 32, 8, 64, ps, 10,
+                                   0.1, None, None) == 2
     # 12 query heads over 8 KV heads
     assert lib.tv_paged_decode(p, p, p, p, p, 4, p, 1, 12, 8, 64, 16, 10,
                                0.1, None, None) == 2

@@ -18,17 +18,18 @@ from oracle.pool import PAGE, PagePool, pages_for
 H, D = 2, 4   # a small pool: 2 KV heads x 4 dims per row
 
 
-def _fresh(num_pages, batch, max_blocks):
+def _fresh(num_pages, batch, max_blocks, page_size=PAGE):
     bt = np.full((batch, max_blocks), -1, np.int64)
     ctx = np.zeros(batch, np.int64)
-    kp = np.zeros((num_pages, PAGE, H, D), np.int64)
-    return PagePool(num_pages), bt, ctx, kp, kp.copy()
+    kp = np.zeros((num_pages, page_size, H, D), np.int64)
+    return (PagePool(num_pages, page_size=page_size), bt, ctx, kp,
+            kp.copy())
 
 
 def _check_conservation(pool, bt, ctx):
     held = np.zeros(pool.num_pages, np.int64)
     for s in range(len(ctx)):
-        for b in range(pages_for(ctx[s])):
+        for b in range(pages_for(ctx[s], pool.ps)):
             held[bt[s][b]] += 1
     np.testing.assert_array_equal(held, pool.ref)
     assert len(set(pool.stack)) == pool.top
@@ -37,7 +38,8 @@ def _check_conservation(pool, bt, ctx):
 
 
 def _gather(kp, bt, s, ctx):
-    return [kp[bt[s][t // PAGE], t % PAGE].copy() for t in range(ctx)]
+    ps = kp.shape[1]
+    return [kp[bt[s][t // ps], t % ps].copy() for t in range(ctx)]
 
 
 def test_fresh_pool_hands_out_pages_in_order_and_maps_slots():
@@ -98,6 +100,14 @@ def test_fork_then_only_the_child_appends():
     _check_conservation(pool, bt, ctx)
 
 
+def test_page_size_32_pops_and_slots():
+    pool, bt, ctx, kp, vp = _fresh(8, 2, 4, page_size=32)
+    slots, _ = pool.append_slots(bt, ctx, [33, 32], kp, vp)
+    assert bt[0][:2].tolist() == [0, 1] and bt[1][:1].tolist() == [2]
+    assert slots.tolist() == list(range(0, 33)) + list(range(64, 96))
+    _check_conservation(pool, bt, ctx)
+
+
 def test_full_shared_pages_are_not_copied():
     pool, bt, ctx, kp, vp = _fresh(8, 2, 4)
     pool.append_slots(bt, ctx, [32, 0], kp, vp)     # two full pages
@@ -108,11 +118,11 @@ def test_full_shared_pages_are_not_copied():
     _check_conservation(pool, bt, ctx)
 
 
-@pytest.mark.parametrize("seed", [1, 2, 3])
-def test_random_operations_match_a_contiguous_cache(seed):
+@pytest.mark.parametrize("seed,page_size", [(1, 16), (2, 16), (3, 32)])
+def test_random_operations_match_a_contiguous_cache(seed, page_size):
     rng = np.random.default_rng(seed)
     batch, max_blocks, num_pages = 12, 24, 200
-    pool, bt, ctx, kp, vp = _fresh(num_pages, batch, max_blocks)
+    pool, bt, ctx, kp, vp = _fresh(num_pages, batch, max_blocks, page_size)
     model = [[] for _ in range(batch)]      # contiguous K rows per sequence
     counter = 1
     for step in range(120):
@@ -120,7 +130,7 @@ def test_random_operations_match_a_contiguous_cache(seed):
         if op < 0.6:
             n = np.where(rng.random(batch) < 0.7,
                          rng.integers(1, 40, batch), 0)
-            n = np.minimum(n, max_blocks * PAGE - ctx)
+            n = np.minimum(n, max_blocks * page_size - ctx)
             before = ctx.copy()
             slots, served = pool.append_slots(bt, ctx, n, kp, vp)
             # write the new rows through the slot mapping
@@ -133,8 +143,9 @@ def test_random_operations_match_a_contiguous_cache(seed):
                     counter += 1
                     sl = slots[k]
                     k += 1
-                    assert sl == bt[s][t // PAGE] * PAGE + t % PAGE
-                    kp[sl // PAGE, sl % PAGE] = row
+                    assert sl == (bt[s][t // page_size] * page_size +
+                                  t % page_size)
+                    kp[sl // page_size, sl % page_size] = row
                     model[s].append(row)
             assert k == len(slots)
         elif op < 0.8:
