@@ -311,6 +311,19 @@ tv_status tv_paged_decode_split_static(
     void* stream);
 
 /*
+ * tv_selftest_wait_timeout -- exercises the bounded wait behind every
+ * TV_DEVERR_TIMEOUT: one thread waits on an mbarrier that nothing completes,
+ * gives up after limit_ns nanoseconds of %globaltimer (clamped to the
+ * library's 2 s), ORs TV_DEVERR_TIMEOUT into *err and returns.  The call
+ * faults nothing and leaves the context usable; it is how the failure path
+ * is tested without a failure.  The pages have no counterpart.
+ *   err        device uint32 word (required)
+ *   waited_ns  device uint64 (nullable): time actually waited
+ */
+tv_status tv_selftest_wait_timeout(uint32_t* err, int64_t limit_ns,
+                                   uint64_t* waited_ns, void* stream);
+
+/*
  * ---- Device page pool -------------------------------------------------------
  * The KV pages of [P3] "内存池管理" as a device-resident pool: a free-page stack
  * and a reference count per page, so that a decode step -- room for the new

@@ -54,6 +54,7 @@ SIGNATURES = {
     "tv_paged_decode_balanced": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
                                       _I, _I, _I, _I, _I64, _F, _P,
                                       ctypes.c_size_t, _P, _P]),
+    "tv_selftest_wait_timeout": (_I, [_P, _I64, _P, _P]),
     "tv_pool_init": (_I, [_P, _I64, _I, _P, _I, _P, _I, _P, _P]),
     "tv_pool_append_slots": (_I, [_P, _I64, _P, _I, _P, _P, _I, _P, _P, _P,
                                   _I, _I, _I, _P, _P]),
@@ -469,3 +470,14 @@ def tv_decode_step(state, out, q, k_new, v_new, k_pool, v_pool, block_tables,
         _ptr(context_lens), b, hq, hkv, d, ps, float(scale), _ptr(workspace),
         workspace.numel() if workspace is not None else 0, _ptr(err),
         _stream(stream)), "tv_decode_step")
+
+
+def tv_selftest_wait_timeout(err, limit_ns, waited_ns=None, stream=None):
+    """Run the bounded-wait self-test (see include/tv.h)."""
+    lib = load()
+    _cuda(err, torch.int32, "err")
+    if waited_ns is not None:
+        _cuda(waited_ns, torch.int64, "waited_ns")
+    _check(lib.tv_selftest_wait_timeout(_ptr(err), int(limit_ns),
+                                        _ptr(waited_ns), _stream(stream)),
+           "tv_selftest_wait_timeout")

@@ -357,6 +357,17 @@ tv_status tv_paged_decode_balanced(void* out, const void* q,
                        &ws);
 }
 
+tv_status tv_selftest_wait_timeout(uint32_t* err, int64_t limit_ns,
+                                   uint64_t* waited_ns, void* stream) {
+  if (!err || limit_ns < 0) return TV_ERR_INVALID_ARG;
+  // never longer than the library's own limit
+  const int64_t lim = limit_ns < 2000000000 ? limit_ns : 2000000000;
+  return cuda_status(tv::launch_wait_selftest(
+      err, (unsigned long long)lim,
+      reinterpret_cast<unsigned long long*>(waited_ns),
+      static_cast<cudaStream_t>(stream)));
+}
+
 // ---- device page pool ---------------------------------------------------------
 
 static tv_status pool_common(const int32_t* pool_state, int64_t num_pages,

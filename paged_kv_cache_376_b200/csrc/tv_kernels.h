@@ -73,6 +73,11 @@ cudaError_t launch_pool_release(int32_t* state, int num_pages, int32_t* bt,
                                 const int32_t* seqs, int num_release,
                                 uint32_t* err, cudaStream_t stream);
 
+// Bounded-wait self-test (selftest.cu).
+cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long limit_ns,
+                                 unsigned long long* waited_ns,
+                                 cudaStream_t stream);
+
 cudaError_t launch_kv_append(const void* k_new, const void* v_new,
                              const int32_t* slot_mapping, int64_t num_tokens,
                              void* k_pool, void* v_pool, int64_t num_slots,
