@@ -27,13 +27,18 @@
 //    A read from tensor memory, so the tensor core's shared-memory reads are
 //    only q, K and V (with P in shared memory the MMAs were starved on
 //    shared-memory bandwidth).  S/P is double-buffered per query tile and
-//    K/V run through an 8-stage ring, so the MMA thread issues S_{j+1} while
-//    tile j is exponentiated and P_j.V_j while tile j+1 is.
+//    K/V run through an 8-stage ring, so S_{j+1} is issued while tile j is
+//    exponentiated and P_j.V_j while tile j+1 is.
 //  * warp 0: TMA producer (q once, K/V ring).
-//    warp 1: tensor-memory allocation and the single MMA-issuing thread:
-//      S_t = Q_t K_j^T (M128 N64 K16 x4) into one of tile t's two S/P
-//      buffers, then O_t += P_t V_j (M128 N64 K16 x4, once for P_hi and once
-//      for P_lo; V read as an MN-major operand) accumulated in tile t's O.
+//    warps 1-3: three MMA-issuing threads.  Warp 3 issues S_t = Q_t K_j^T
+//      (M128 N64 K16 x4) for both tiles into one of tile t's two S/P
+//      buffers; warp 1 / warp 2 issue O_t += P_t V_j for tile A / B (M128
+//      N64 K16 x4, once for P_hi and once for P_lo; V read as an MN-major
+//      operand) accumulated in tile t's O.  Issuing a tcgen05.mma takes its
+//      thread several times longer than the tensor core needs for one of
+//      these small products, so a single issuer left the tensor core idle
+//      most of the time; three independent instruction streams keep it fed.
+//      Warp 1 also allocates the tensor memory.
 //    warps 4-7 / 8-11: softmax of tile A / B.  Thread = one MMA row = one
 //      (query, head).  It reads its 64 scores from tensor memory in one load,
 //      takes their maximum, moves the running maximum only when it grows by
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.q_full), 1);
     for (int i = 0; i < kST; ++i) {
       mbar_init(smem_u32(&sm.kv_full[i]), 1);
-      mbar_init(smem_u32(&sm.kv_empty[i]), 1);
+      mbar_init(smem_u32(&sm.kv_empty[i]), 3);   // three issuers
     }
     for (int t = 0; t < kQTiles; ++t) {
       for (int b = 0; b < 2; ++b) {
@@ -202,69 +207,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer =======================================
+  } else if (warp >= 1 && warp <= 3) {
+    // ======================= MMA issuers ======================================
+    // warp 3 issues S = Q K^T for both query tiles; warps 1 / 2 issue
+    // O += P V for tile A / B.  A tcgen05.mma costs its issuing thread far
+    // more time than the tensor core needs for an M128 N64 K16 product, so
+    // the three instruction streams run in parallel.  tcgen05.commit tracks
+    // only the committing thread's own MMAs, so every issuer signals its own
+    // barriers; the K/V stage of tile j is free after all three arrived.
+    // Barrier X[t][b] serves the tiles j with j % 2 == b; its (j / 2)-th
+    // phase belongs to tile j, so a wait for tile j uses parity (j >> 1) & 1.
     if (lane == 0) {
-      bool ok = mbar_wait(smem_u32(&sm.q_full), 0);
-      // Barrier X[t][b] serves the tiles j with j % 2 == b; its (j / 2)-th
-      // phase belongs to tile j, so a wait for tile j uses parity (j >> 1) & 1.
-      auto issue_qk = [&](int t, int j) -> bool {
-        const int b = j & 1;
-        // S/P buffer b holds P of tile j - 2 until its P.V has completed
-        if (j >= 2 &&
-            !mbar_wait(smem_u32(&sm.o_done[t][b]), ((j - 2) >> 1) & 1))
-          return false;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm.q[t]);
-        const uint32_t k_addr = smem_u32(sm.k[j % kST]);
-#pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
-          const uint64_t ad = smem_desc_sw128(q_addr + k * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(k_addr + k * 32, 16, 1024);
-          tc_mma_bf16(tmem + kSCol + (2 * t + b) * kBN, ad, bd, kIdescQK,
-                      k > 0);
-        }
-        tc_commit(smem_u32(&sm.s_full[t][b]));
-        return true;
-      };
-      auto issue_pv = [&](int t, int j) -> bool {
-        const int b = j & 1;
-        if (!mbar_wait(smem_u32(&sm.p_full[t][b]), (j >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.v[j % kST]);
-        const uint32_t p_col = tmem + kSCol + (2 * t + b) * kBN;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
-#pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            // A = P in tensor memory: keys [16k, 16k+16) = 8 columns
-            const uint32_t a_tmem = p_col + part * (kBN / 2) + k * 8;
-            // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
-            const uint64_t bd =
-                smem_desc_sw128(v_addr + k * 16 * kRowBytes, kTileBytes, 1024);
-            tc_mma_bf16_ts(tmem + kOCol + t * kD, a_tmem, bd, kIdescPV,
-                           (j | part | k) != 0);
-          }
-        }
-        tc_commit(smem_u32(&sm.o_done[t][b]));
-        return true;
-      };
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
+      bool ok = true;
+      if (warp == 3) {
+        ok = mbar_wait(smem_u32(&sm.q_full), 0);
+        for (int j = 0; ok && j < n_tiles; ++j) {
           if (!mbar_wait(smem_u32(&sm.kv_full[j % kST]), (j / kST) & 1)) {
             ok = false;
             break;
           }
-        }
-        // S for tile j, P.V for tile j - 1, interleaving the two query tiles
+          const int b = j & 1;
+          bool any = false;
 #pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-          if (ok && j < n_tiles_of[t] && !issue_qk(t, j)) ok = false;
-          if (ok && j >= 1 && j - 1 < n_tiles_of[t] && !issue_pv(t, j - 1))
-            ok = false;
+          for (int t = 0; t < kQTiles; ++t) {
+            if (j >= n_tiles_of[t]) continue;
+            // S/P buffer b holds P of tile j - 2 until its P.V has completed
+            if (j >= 2 &&
+                !mbar_wait(smem_u32(&sm.o_done[t][b]), ((j - 2) >> 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(sm.q[t]);
+            const uint32_t k_addr = smem_u32(sm.k[j % kST]);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(q_addr + k * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(k_addr + k * 32, 16, 1024);
+              tc_mma_bf16(tmem + kSCol + (2 * t + b) * kBN, ad, bd, kIdescQK,
+                          k > 0);
+            }
+            tc_commit(smem_u32(&sm.s_full[t][b]));
+            any = true;
+          }
+          if (!ok) break;
+          if (any) tc_commit(smem_u32(&sm.kv_empty[j % kST]));
+          else mbar_arrive(smem_u32(&sm.kv_empty[j % kST]));
         }
-        if (!ok) break;
-        if (j >= 1) tc_commit(smem_u32(&sm.kv_empty[(j - 1) % kST]));
+      } else {
+        const int t = warp - 1;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int st = j % kST;
+          // every issuer waits for tile j's stage before releasing it, so
+          // that no issuer arrives twice in one phase of kv_empty
+          if (!mbar_wait(smem_u32(&sm.kv_full[st]), (j / kST) & 1)) {
+            ok = false;
+            break;
+          }
+          if (j < n_tiles_of[t]) {
+            const int b = j & 1;
+            // P of tile j is in tensor memory; where tile A's softmax zeroes
+            // stale V rows of this key tile, tile B's P.V also waits for it
+            const int key0 = j * kBN;
+            const bool zeroed = max(ctx, key0) < min(n_pages * kPS, key0 + kBN);
+            if (!mbar_wait(smem_u32(&sm.p_full[t][b]), (j >> 1) & 1) ||
+                (t == 1 && zeroed && j < n_tiles_of[0] &&
+                 !mbar_wait(smem_u32(&sm.p_full[0][b]), (j >> 1) & 1))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(sm.v[st]);
+            const uint32_t p_col = tmem + kSCol + (2 * t + b) * kBN;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {          // P_hi, then P_lo
+#pragma unroll
+              for (int k = 0; k < kBN / 16; ++k) {
+                // A = P in tensor memory: keys [16k, 16k+16) = 8 columns
+                const uint32_t a_tmem = p_col + part * (kBN / 2) + k * 8;
+                // B = V: MN-major (head dim contiguous); 16 keys = 2 x 8 rows
+                const uint64_t bd = smem_desc_sw128(v_addr + k * 16 * kRowBytes,
+                                                    kTileBytes, 1024);
+                tc_mma_bf16_ts(tmem + kOCol + t * kD, a_tmem, bd, kIdescPV,
+                               (j | part | k) != 0);
+              }
+            }
+            tc_commit(smem_u32(&sm.o_done[t][b]));
+            tc_commit(smem_u32(&sm.kv_empty[st]));
+          } else {
+            mbar_arrive(smem_u32(&sm.kv_empty[st]));
+          }
+        }
       }
       if (!ok) flag_error(a.err, DEVERR_TIMEOUT);
     }
@@ -339,23 +372,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
 
       // ---- exponentials, row sum, P_hi / P_lo back into the S columns ------------
-      float lsum = 0.f;
+      // packed fp32x2 arithmetic: one instruction per pair of keys
+      float2 lsum2 = make_float2(0.f, 0.f);
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      const float2 neg1 = make_float2(-1.f, -1.f);
       uint32_t hi[kBN / 2], lo[kBN / 2];
 #pragma unroll
       for (int e = 0; e < kBN / 2; ++e) {
-        const float x0 = fast_exp2(fmaf(s[2 * e], c, -m_use));
-        const float x1 = fast_exp2(fmaf(s[2 * e + 1], c, -m_use));
-        lsum += x0 + x1;
-        hi[e] = pack_bf16x2(x0, x1);
-        lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+        const float2 t = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), c2,
+                                    nm2);
+        const float2 x = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        lsum2 = __fadd2_rn(lsum2, x);
+        hi[e] = pack_bf16x2(x.x, x.y);
+        const float2 h = make_float2(bf16_lo(hi[e]), bf16_hi(hi[e]));
+        const float2 r = __ffma2_rn(h, neg1, x);   // x - hi, exact
+        lo[e] = pack_bf16x2(r.x, r.y);
       }
+      const float lsum = lsum2.x + lsum2.y;
       tmem_st32(s_addr + b * kBN, hi);
       tmem_st32(s_addr + b * kBN + kBN / 2, lo);
       l_run += lsum;
 
       // ---- keys past the context in a loaded page may hold stale data: zero
-      //      their V rows (once per key tile, by the query tile whose P.V on
-      //      it is issued first) so that P = 0 cannot meet NaN in the MMA ----
+      //      their V rows (once per key tile: by tile A where it has this
+      //      key tile, else by B; tile B's P.V on a key tile that A zeroes
+      //      waits for A's P as well) so that P = 0 cannot meet NaN ----
       if (t == 0 || j >= n_tiles_of[0]) {
         const int z0 = max(ctx, key0);
         const int z1 = min(n_pages * kPS, key0 + kBN);
