@@ -123,7 +123,8 @@ def _config(wl, name, kind=None, engine=False):
                        "tv_split_merge")
         cfg["partition_tokens"] = wl.partition_tokens
     else:
-        cfg["step"] = "tv_kv_append (512-token chunks) + tv_paged_prefill"
+        cfg["step"] = ("tv_kv_append (512-token chunks) + tv_paged_prefill "
+                       "(cost-ordered dispatch)")
         cfg["query_rows"] = int(wl.q.shape[0])
     if engine:
         cfg["step"] = ("tv_decode_step: device page pool slot reservation, "
@@ -232,6 +233,8 @@ class TVRunner:
                                   device=device)
             self.maxp = maxp
         self.maxq = int(np.diff(wl.query_start_loc).max())
+        if self.kind == "prefill":
+            self.pws = _lib.prefill_workspace(wl.num_seqs, self.maxq, device)
         self.stream = torch.cuda.current_stream(device)
         self.engine = engine
         if engine:
@@ -355,7 +358,8 @@ class TVRunner:
                 self._p(db.query_start_loc), self._p(db.k_pool),
                 self._p(db.v_pool), self._p(db.block_tables), mb,
                 self._p(db.context_lens), b, self.maxq, hq, hkv, d, ps,
-                num_pages, wl.scale, self._p(db.err), s)
+                num_pages, wl.scale, self._p(self.pws), self.pws.numel(),
+                self._p(db.err), s)
         assert st == 0, st
         if timing is not None:
             timing[1].record(self.stream)
@@ -369,7 +373,9 @@ class TVRunner:
     def launches_per_step(self):
         if self.engine:
             return 2
-        return {"split": 3, "fused": 1, "balanced": 1}.get(self.kind, 2)
+        # prefill: append, the dispatch-order kernel, attention
+        return {"split": 3, "fused": 1, "balanced": 1,
+                "prefill": 3}.get(self.kind, 2)
 
     def graph_timed(self):
         """Steps timed by CUDA-graph replay: one launch per step, or the

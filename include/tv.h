@@ -257,14 +257,27 @@ tv_status tv_split_merge(void* out, const float* partial_out,
  * their K,V must already be in the cache (tv_kv_append).  With T_s rows and
  * C = context_lens[s], row i sits at position C - T_s + i and attends to
  * keys 0 .. C - T_s + i.  QK^T and PV run on the tcgen05 tensor cores (bf16
- * in, fp32 accumulate in tensor memory); P is rounded to bf16 for PV.
+ * in, fp32 accumulate in tensor memory); P enters PV as the sum of two bf16
+ * terms (p rounded, plus the rounding remainder).
  *   out              [total_rows][num_q_heads][head_dim] bf16, written
  *   q                [total_rows][num_q_heads][head_dim] bf16
  *   num_query_rows   total_rows (the row count of q and out)
  *   query_start_loc  [num_seqs + 1] int32, non-decreasing, [0] == 0,
  *                    [num_seqs] <= num_query_rows
  *   max_query_len    >= every T_s (sizes the grid); rows beyond a
- *                    sequence's T_s are not touched
+ *                    sequence's T_s are not touched; at most 65535 * 64
+ *   workspace        NULL, or device memory of at least
+ *                    tv_prefill_workspace_size() bytes, 16-byte aligned, no
+ *                    initial contents needed; too small or misaligned
+ *                    returns TV_ERR_INVALID_ARG.  Given, a one-CTA kernel
+ *                    first lists the work blocks (64 query rows of one
+ *                    sequence) by their number of key tiles, costliest
+ *                    first, and the attention grid runs them in that order,
+ *                    so that long-context blocks do not start last and hold
+ *                    a few SMs while the rest idle.  The results are the
+ *                    same with and without it.  Concurrent calls need
+ *                    separate workspaces.
+ *   workspace_bytes  its size
  * A sequence with T_s > C is flagged TV_DEVERR_BAD_QUERY and skipped.
  */
 tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
@@ -273,8 +286,18 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
                            int max_blocks_per_seq, const int32_t* context_lens,
                            int num_seqs, int max_query_len, int num_q_heads,
                            int num_kv_heads, int head_dim, int page_size,
-                           int64_t num_pages, float scale, uint32_t* err,
+                           int64_t num_pages, float scale, void* workspace,
+                           size_t workspace_bytes, uint32_t* err,
                            void* stream);
+
+/*
+ * tv_prefill_workspace_size -- bytes of the optional tv_paged_prefill
+ * workspace for num_seqs sequences and the given max_query_len (4 bytes per
+ * 64-row block of every sequence, rounded up to 16).
+ *   bytes   host pointer, written on TV_OK
+ */
+tv_status tv_prefill_workspace_size(int num_seqs, int max_query_len,
+                                    size_t* bytes);
 
 /*
  * tv_paged_decode_split_static -- tv_paged_decode_split followed by

@@ -45,7 +45,10 @@ SIGNATURES = {
                                    _I, _I, _I, _I64, _F, _I, _I, _P, _P]),
     "tv_split_merge": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "tv_paged_prefill": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _P, _I, _I,
-                              _I, _I, _I, _I, _I64, _F, _P, _P]),
+                              _I, _I, _I, _I, _I64, _F, _P, ctypes.c_size_t,
+                              _P, _P]),
+    "tv_prefill_workspace_size": (_I, [_I, _I,
+                                       ctypes.POINTER(ctypes.c_size_t)]),
     "tv_paged_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I,
                                           _I, _I, _I, _I64, _F, _I, _I, _P,
                                           _P]),
@@ -240,11 +243,28 @@ def tv_split_merge(out, partial_out, partial_lse, context_lens,
         "tv_split_merge")
 
 
+def tv_prefill_workspace_size(num_seqs, max_query_len):
+    n = ctypes.c_size_t(0)
+    _check(load().tv_prefill_workspace_size(int(num_seqs), int(max_query_len),
+                                            ctypes.byref(n)),
+           "tv_prefill_workspace_size")
+    return n.value
+
+
+def prefill_workspace(num_seqs, max_query_len, device="cuda"):
+    """Device workspace for the cost-ordered prefill dispatch (no initial
+    contents needed)."""
+    n = tv_prefill_workspace_size(num_seqs, max_query_len)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
 def tv_paged_prefill(out, q, query_start_loc, k_pool, v_pool, block_tables,
                      context_lens, scale, max_query_len, err=None,
-                     stream=None):
+                     stream=None, workspace=None, ordered=True):
     """out[rows][Hq][D] (bf16) = chunked-prefill attention of q[rows][Hq][D]
-    over the paged cache (chunk K/V already appended)."""
+    over the paged cache (chunk K/V already appended).  With ordered=True
+    the blocks run costliest first, through ``workspace`` (allocated here
+    when None); ordered=False keeps grid order (same results)."""
     lib = load()
     bf = torch.bfloat16
     for n, t in (("out", out), ("q", q), ("k_pool", k_pool),
@@ -260,12 +280,18 @@ def tv_paged_prefill(out, q, query_start_loc, k_pool, v_pool, block_tables,
     b = context_lens.shape[0]
     if out.shape != q.shape or query_start_loc.shape != (b + 1,):
         raise ValueError("shape mismatch")
+    ws, ws_bytes = None, 0
+    if ordered:
+        if workspace is None:
+            workspace = prefill_workspace(b, max_query_len, q.device)
+        _cuda(workspace, workspace.dtype, "workspace")
+        ws, ws_bytes = workspace, workspace.numel() * workspace.element_size()
     _check(lib.tv_paged_prefill(
         _ptr(out), _ptr(q), rows, _ptr(query_start_loc), _ptr(k_pool),
         _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
         _ptr(context_lens), b, int(max_query_len), hq, hkv, d, page_size,
-        num_pages, float(scale), _ptr(err), _stream(stream)),
-        "tv_paged_prefill")
+        num_pages, float(scale), _ptr(ws), ws_bytes, _ptr(err),
+        _stream(stream)), "tv_paged_prefill")
 
 
 def tv_paged_decode_split_static(out, q, k_pool, v_pool, block_tables,

@@ -90,6 +90,82 @@ struct PrefillSmem {
   uint32_t bad_pages[kST];
 };
 
+// ---- dispatch order ------------------------------------------------------------
+// The cost of a CTA is its number of key tiles, (P + last row + 1) / 64 rounded
+// up, so within one launch CTAs differ by up to the longest context / 64 tiles.
+// Dispatched in grid order, the costliest can start last and hold a few SMs
+// while the rest idle.  This kernel (one CTA) lists the (sequence, block) items
+// costliest first by a counting sort: a histogram of the costs in shared memory,
+// an exclusive scan in descending cost order, then every item takes the next
+// slot of its cost.  Items of equal cost land in an unspecified order; the
+// prefill's results do not depend on the order, only its timing does.
+constexpr int kOrderThreads = 1024;
+constexpr int kCostBuckets = 4096;                // costs above share the top
+constexpr int kBucketsPerThread = kCostBuckets / kOrderThreads;
+
+__device__ __forceinline__ int prefill_cost(const PrefillArgs& a, int item,
+                                            int nblk) {
+  const int seq = item / nblk;
+  const int blk = item - seq * nblk;
+  const int T = a.query_start_loc[seq + 1] - a.query_start_loc[seq];
+  const int ctx = min(a.context_lens[seq],
+                      a.max_blocks_per_seq * (kPS << a.page_shift));
+  const int q0 = blk * kPrefillRowsPerCta;
+  if (T <= 0 || q0 >= T || T > ctx) return 0;    // no work (or flagged)
+  const int tiles =
+      (ctx - T + min(q0 + kPrefillRowsPerCta, T) + kBN - 1) / kBN;
+  return min(tiles, kCostBuckets - 1);
+}
+
+__global__ void __launch_bounds__(kOrderThreads, 1)
+    prefill_order_kernel(const PrefillArgs a) {
+  __shared__ int slot[kCostBuckets];   // histogram, then next free position
+  __shared__ int warp_sum[kOrderThreads / 32];
+  const int nblk = prefill_blocks(a.max_query_len);
+  const int n = a.num_seqs * nblk;
+  for (int i = threadIdx.x; i < kCostBuckets; i += kOrderThreads) slot[i] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kOrderThreads)
+    atomicAdd(&slot[prefill_cost(a, i, nblk)], 1);
+  __syncthreads();
+  // thread t owns the buckets of costs kCostBuckets-1-4t down to ...-4t-3
+  int own[kBucketsPerThread];
+  int sum = 0;
+#pragma unroll
+  for (int k = 0; k < kBucketsPerThread; ++k) {
+    own[k] = slot[kCostBuckets - 1 - (threadIdx.x * kBucketsPerThread + k)];
+    sum += own[k];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sum[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += v;
+    }
+    warp_sum[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  int start = incl - sum + (warp > 0 ? warp_sum[warp - 1] : 0);
+#pragma unroll
+  for (int k = 0; k < kBucketsPerThread; ++k) {
+    slot[kCostBuckets - 1 - (threadIdx.x * kBucketsPerThread + k)] = start;
+    start += own[k];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kOrderThreads)
+    a.order[atomicAdd(&slot[prefill_cost(a, i, nblk)], 1)] = i;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const PrefillArgs a,
                          const __grid_constant__ CUtensorMap tm_q,
@@ -100,8 +176,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto& sm = *reinterpret_cast<PrefillSmem*>(base);
 
   const int kvh = blockIdx.x;
-  const int blk = gridDim.y - 1 - blockIdx.y;    // heaviest blocks first
-  const int seq = blockIdx.z;
+  int blk = gridDim.y - 1 - blockIdx.y;    // heaviest blocks of a sequence first
+  int seq = blockIdx.z;
+  if (a.order) {                           // costliest (sequence, block) first
+    const int item = a.order[blockIdx.y + gridDim.y * blockIdx.z];
+    seq = item / gridDim.y;
+    blk = item - seq * gridDim.y;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -460,8 +541,13 @@ cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,
   cudaError_t e = cudaFuncSetAttribute(
       paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int blocks = (a.max_query_len + kQRows * kQTiles - 1) /
-                     (kQRows * kQTiles);
+  static_assert(kQRows * kQTiles == kPrefillRowsPerCta, "rows per CTA");
+  if (a.order) {
+    prefill_order_kernel<<<1, kOrderThreads, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int blocks = prefill_blocks(a.max_query_len);
   dim3 grid(a.num_kv_heads, blocks, a.num_seqs);
   paged_prefill_kernel<<<grid, kThreads, smem, stream>>>(a, tq, tk, tv);
   return cudaGetLastError();

@@ -527,13 +527,26 @@ tv_status tv_split_merge(void* out, const float* partial_out,
       static_cast<cudaStream_t>(stream)));
 }
 
+static size_t prefill_workspace_bytes(int num_seqs, int max_query_len) {
+  const size_t items = (size_t)num_seqs * (size_t)tv::prefill_blocks(max_query_len);
+  return (items * sizeof(int32_t) + 15) / 16 * 16;
+}
+
+tv_status tv_prefill_workspace_size(int num_seqs, int max_query_len,
+                                    size_t* bytes) {
+  if (!bytes || num_seqs < 0 || max_query_len < 0) return TV_ERR_INVALID_ARG;
+  *bytes = prefill_workspace_bytes(num_seqs, max_query_len);
+  return TV_OK;
+}
+
 tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
                            const int32_t* query_start_loc, const void* k_pool,
                            const void* v_pool, const int32_t* block_tables,
                            int max_blocks_per_seq, const int32_t* context_lens,
                            int num_seqs, int max_query_len, int num_q_heads,
                            int num_kv_heads, int head_dim, int page_size,
-                           int64_t num_pages, float scale, uint32_t* err,
+                           int64_t num_pages, float scale, void* workspace,
+                           size_t workspace_bytes, uint32_t* err,
                            void* stream) {
   tv_status st =
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
@@ -552,8 +565,11 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) ||
       !aligned16(v_pool))
     return TV_ERR_INVALID_ARG;
-  const int64_t grid_x = (int64_t)(max_query_len + 31) / 32 * num_kv_heads;
-  if (grid_x > INT32_MAX) return TV_ERR_UNSUPPORTED;
+  if (workspace &&
+      (!aligned16(workspace) ||
+       workspace_bytes < prefill_workspace_bytes(num_seqs, max_query_len)))
+    return TV_ERR_INVALID_ARG;
+  if (tv::prefill_blocks(max_query_len) > 65535) return TV_ERR_UNSUPPORTED;
 
   // Query rows past num_query_rows read as zeros and are never stored.
   CUtensorMap tq, tk, tvm;
@@ -582,6 +598,7 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   a.num_query_rows = num_query_rows;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.page_shift = page_shift(page_size);
+  a.order = static_cast<int32_t*>(workspace);
   return cuda_status(tv::launch_paged_prefill(
       a, tq, tk, tvm, static_cast<cudaStream_t>(stream)));
 }

@@ -105,8 +105,18 @@ struct PrefillArgs {
   int64_t num_query_rows;
   float scale_log2;
   int page_shift;                // page_size = 16 << page_shift
+  // Dispatch order: order[i] = seq * prefill_blocks(max_query_len) + block of
+  // the i-th CTA group (costliest first), written by the ordering kernel
+  // into caller workspace; nullptr = grid order.
+  int32_t* order;
 };
 
+constexpr int kPrefillRowsPerCta = 64;   // query rows (chunk positions) per CTA
+__host__ __device__ inline int prefill_blocks(int max_query_len) {
+  return (max_query_len + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
+}
+
+// Launches the ordering kernel first when a.order is set.
 cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,
                                  const CUtensorMap& tk, const CUtensorMap& tv,
                                  cudaStream_t stream);

@@ -67,7 +67,7 @@ def test_unsupported_shapes_are_rejected_before_launch(lib):
     assert lib.tv_split_merge(p, p, p, p, 2, 32, 32, 512, 4, None) == 2
     # prefill needs 4 query heads per KV head
     assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, 4, p, 1, 8, 8, 8, 64,
-                                16, 10, 0.1, None, None) == 2
+                                16, 10, 0.1, None, 0, None, None) == 2
 
 
 def test_invalid_arguments_are_rejected_before_launch(lib):
@@ -89,6 +89,25 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
     assert lib.tv_kv_append(p, p, p, -1, p, p, 10, 8, 64, 16, None,
                             None) == 1
     assert lib.tv_split_merge(None, p, p, p, 2, 32, 64, 512, 4, None) == 1
+    # prefill workspace too small for 3 sequences x 2 blocks, or misaligned
+    assert lib.tv_paged_prefill(p, p, 100, p, p, p, p, 4, p, 3, 100, 32, 8,
+                                64, 16, 10, 0.1, p, 16, None, None) == 1
+    assert lib.tv_paged_prefill(p, p, 100, p, p, p, p, 4, p, 3, 100, 32, 8,
+                                64, 16, 10, 0.1, unaligned, 64, None,
+                                None) == 1
+
+
+def test_prefill_workspace_size(lib):
+    import ctypes
+    n = ctypes.c_size_t(0)
+    # 4 bytes per 64-row block of every sequence, rounded up to 16
+    assert lib.tv_prefill_workspace_size(3, 100, ctypes.byref(n)) == 0
+    assert n.value == 32          # 3 x 2 blocks = 24 bytes
+    assert lib.tv_prefill_workspace_size(16, 512, ctypes.byref(n)) == 0
+    assert n.value == 512         # 16 x 8 blocks
+    assert lib.tv_prefill_workspace_size(0, 0, ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert lib.tv_prefill_workspace_size(-1, 8, ctypes.byref(n)) == 1
 
 
 def test_empty_work_is_a_no_op(lib):
@@ -98,8 +117,8 @@ def test_empty_work_is_a_no_op(lib):
     assert lib.tv_paged_decode(None, None, None, None, None, 4, None, 0, 32,
                                8, 64, 16, 10, 0.1, None, None) == 0
     assert lib.tv_paged_prefill(None, None, 0, None, None, None, None, 4,
-                                None, 0, 0, 32, 8, 64, 16, 10, 0.1, None,
-                                None) == 0
+                                None, 0, 0, 32, 8, 64, 16, 10, 0.1, None, 0,
+                                None, None) == 0
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):

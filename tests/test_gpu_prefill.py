@@ -110,3 +110,34 @@ def test_physical_page_permutation_is_bit_identical():
         db = upload(wl)
         outs.append(bf16_bits(gpu_prefill(db, wl.scale, 70)))
     np.testing.assert_array_equal(outs[0], outs[1])
+
+
+def test_cost_ordered_dispatch_is_bit_identical_to_grid_order():
+    """The dispatch order changes only which CTA runs when: both orders give
+    the same bits, and both match the oracle.  Prefixes of very different
+    lengths make the cost order differ from the grid order; one sequence has
+    fewer rows than max_query_len (blocks with no work sort last), and the
+    workspace is filled with garbage first (it needs no initial contents)."""
+    from paged_kv_cache_376_b200 import _lib
+    wl = W.prefill_workload([3000, 0, 17, 1500, 64, 4000],
+                            [100, 257, 64, 31, 190, 65], seed=77)
+    db = upload(wl)
+    gpu_append(db)
+    maxq = int(np.diff(wl.query_start_loc).max())
+    outs = []
+    for ordered in (False, True):
+        out = torch.full_like(db.q, float("nan"))
+        ws = _lib.prefill_workspace(wl.num_seqs, maxq)
+        ws.fill_(0xA5)
+        _lib.tv_paged_prefill(out, db.q, db.query_start_loc, db.k_pool,
+                              db.v_pool, db.block_tables, db.context_lens,
+                              wl.scale, maxq, err=db.err, workspace=ws,
+                              ordered=ordered)
+        torch.cuda.synchronize()
+        outs.append(out)
+    np.testing.assert_array_equal(bf16_bits(outs[0]), bf16_bits(outs[1]))
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp,
+                               wl.block_tables, wl.context_lens, wl.scale)
+    assert_parity(outs[1], ref, "cost-ordered prefill")
+    assert err_word(db) == 0
