@@ -117,3 +117,15 @@ def test_prefill_config_names_the_ordered_step():
     cfg = bench._config(wl, "prefill")
     assert "tv_paged_prefill" in cfg["step"] and "ordered" in cfg["step"]
     assert cfg["query_rows"] == int(np.asarray(wl.q).shape[0])
+
+
+def test_cpu_baseline_reports_all_cores_and_one_core():
+    import oracle
+    wl = W.tiny_decode()
+    cores = oracle.max_threads()
+    r = bench.cpu_baseline(wl, "tiny", budget_s=0.3)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s"
+    assert r["cores"] == cores and r["value"] > 0
+    one = r["single_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == "GB/s"
+    assert oracle.max_threads() == cores        # thread count restored
