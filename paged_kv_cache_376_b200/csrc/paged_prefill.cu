@@ -51,6 +51,10 @@
 //    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
 //    operands); a single bf16 P carries 8 bits, which is not enough for rows
 //    that see few keys.
+//  * With a workspace, a one-CTA kernel first lists the (sequence, 64-row
+//    block) items costliest first (cost = key tiles), and the attention grid
+//    takes its work from that list, so that the longest blocks do not start
+//    last and hold a few SMs while the rest idle.
 //  * Every wait is an mbarrier wait bounded by a 2 s time limit.
 #include "tv_device.cuh"
 #include "tv_kernels.h"
