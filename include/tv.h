@@ -37,8 +37,10 @@
  *     tokens; the kernels stream 16-token blocks, two per 32-token page),
  *     num_q_heads a multiple of
  *     num_kv_heads with a ratio in {1, 2, 4, 8}; every pointer 16-byte
- *     aligned.  Anything else returns TV_ERR_UNSUPPORTED or
- *     TV_ERR_INVALID_ARG before any launch.
+ *     aligned; num_seqs <= 65535; num_pages * page_size and
+ *     max_blocks_per_seq * page_size at most INT32_MAX (token positions and
+ *     pool rows are 32-bit in the kernels).  Anything else returns
+ *     TV_ERR_UNSUPPORTED or TV_ERR_INVALID_ARG before any launch.
  *   - `err` (nullable) is a device uint32 word; kernels OR bits into it when
  *     they meet bad data and skip that data instead of faulting:
  *       TV_DEVERR_BAD_SLOT     slot_mapping entry >= num_pages * page_size

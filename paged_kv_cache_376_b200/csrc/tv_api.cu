@@ -210,7 +210,10 @@ static tv_status decode_common(void* out, float* partial_out,
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
       !std::isfinite(scale))
     return TV_ERR_INVALID_ARG;
-  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX)
+  // the kernels hold token positions (up to max_blocks_per_seq * page_size)
+  // and pool rows in 32-bit integers
+  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX ||
+      (int64_t)max_blocks_per_seq * page_size > INT32_MAX)
     return TV_ERR_UNSUPPORTED;
   if (split && (partition_tokens <= 0 || partition_tokens % page_size ||
                 max_partitions <= 0 || max_partitions > 65535))
@@ -555,7 +558,8 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
       max_query_len < 0 || num_query_rows < 0 || !std::isfinite(scale))
     return TV_ERR_INVALID_ARG;
-  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX)
+  if (num_seqs > 65535 || num_pages * page_size > INT32_MAX ||
+      (int64_t)max_blocks_per_seq * page_size > INT32_MAX)
     return TV_ERR_UNSUPPORTED;
   if (num_seqs == 0 || max_query_len == 0 || num_query_rows == 0)
     return TV_OK;
@@ -570,6 +574,10 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
        workspace_bytes < prefill_workspace_bytes(num_seqs, max_query_len)))
     return TV_ERR_INVALID_ARG;
   if (tv::prefill_blocks(max_query_len) > 65535) return TV_ERR_UNSUPPORTED;
+  // the ordering kernel counts the (sequence, block) items in an int
+  if (workspace &&
+      (int64_t)num_seqs * tv::prefill_blocks(max_query_len) > INT32_MAX)
+    return TV_ERR_UNSUPPORTED;
 
   // Query rows past num_query_rows read as zeros and are never stored.
   CUtensorMap tq, tk, tvm;

@@ -97,6 +97,22 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
                                 None) == 1
 
 
+def test_sizes_beyond_32_bit_positions_are_refused(lib):
+    p = _fake()
+    big_mb = 1 << 27          # x 16-token pages = 2^31 token positions
+    assert lib.tv_paged_decode(p, p, p, p, p, big_mb, p, 1, 32, 8, 64, 16, 10,
+                               0.1, None, None) == 2
+    assert lib.tv_paged_decode_append(p, p, p, p, p, p, p, big_mb, p, 1, 32,
+                                      8, 64, 16, 10, 0.1, None, None) == 2
+    assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, big_mb, p, 1, 8, 32, 8,
+                                64, 16, 10, 0.1, None, 0, None, None) == 2
+    # 65535 sequences x 65535 blocks of 64 rows: more ordering items than an
+    # int holds (refused only when the ordering workspace is given)
+    assert lib.tv_paged_prefill(p, p, 1 << 30, p, p, p, p, 4, p, 65535,
+                                65535 * 64, 32, 8, 64, 16, 10, 0.1, p,
+                                1 << 40, None, None) == 2
+
+
 def test_prefill_workspace_size(lib):
     import ctypes
     n = ctypes.c_size_t(0)
