@@ -281,11 +281,13 @@ def test_prefill_without_prefix_is_causal_self_attention():
         np.testing.assert_allclose(got[rows], want, rtol=1e-11, atol=1e-12)
 
 
-def test_prefill_with_prefix_matches_brute_force():
+@pytest.mark.parametrize("hq,hkv,d,ps", [(32, 8, 64, 16), (32, 8, 64, 32),
+                                         (8, 2, 8, 4)])
+def test_prefill_with_prefix_matches_brute_force(hq, hkv, d, ps):
     rng = np.random.default_rng(23)
     prefixes, chunks = [0, 5, 33, 100], [3, 20, 16, 9]
     k_seqs, v_seqs, kp, vp, bt, q, qsl, ctx = _prefill_case(
-        rng, prefixes, chunks)
+        rng, prefixes, chunks, hq, hkv, d, ps)
     got = oracle.paged_prefill(q, qsl, kp, vp, bt, ctx, 0.125)
     for s, (p, c) in enumerate(zip(prefixes, chunks)):
         vis = np.arange(p + c)[None, :] <= (p + np.arange(c))[:, None]
