@@ -90,6 +90,7 @@ struct PrefillSmem {
   alignas(8) uint64_t q_full;
   uint64_t kv_full[kST], kv_empty[kST];
   uint64_t s_full[kQTiles][2], p_full[kQTiles][2], o_done[kQTiles][2];
+  uint64_t drain[3];   // error path: each MMA issuer's own MMAs have finished
   uint32_t tmem_base;
   uint32_t bad_pages[kST];
 };
@@ -234,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&sm.o_done[t][b]), 1);
       }
     }
+    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&sm.drain[i]), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -260,6 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= kST &&
             !mbar_wait(smem_u32(&sm.kv_empty[st]), ((j / kST) + 1) & 1)) {
           flag_error(a.err, DEVERR_TIMEOUT);
+          // before giving up, let the copies this thread issued land
+          // (bounded waits): the last tile of every stage, then q
+          for (int jl = j - kST; jl < j; ++jl)
+            mbar_wait(smem_u32(&sm.kv_full[jl % kST]), (jl / kST) & 1);
+          mbar_wait(smem_u32(&sm.q_full), 0);
           break;
         }
         uint32_t bad = 0;
@@ -384,7 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) flag_error(a.err, DEVERR_TIMEOUT);
+      if (!ok) {
+        flag_error(a.err, DEVERR_TIMEOUT);
+        // before giving up, let this thread's MMAs finish (bounded wait), so
+        // that none still writes tensor memory when it is freed
+        tc_commit(smem_u32(&sm.drain[warp - 1]));
+        mbar_wait(smem_u32(&sm.drain[warp - 1]), 0);
+      }
     }
   } else if (warp >= 4) {
     // ======================= softmax warpgroups ===============================
