@@ -90,6 +90,18 @@ def _traffic(kernel, workload_name):
         return None
 
 
+def _roofline_peak(unit, wall_s, hbm, tfl_burst, tfl_sustained):
+    """(peak, bound, MEASURED_PEAKS key) for the dominant kernel: HBM for
+    byte-bound work; for tensor-bound work the sustained GEMM figure when the
+    timed region lasted SUSTAINED_S or more (it then runs under the 1 kW power
+    cap, as that figure was measured), else the burst figure."""
+    if unit == "GB/s":
+        return hbm, "hbm", "hbm_gbs"
+    if wall_s >= SUSTAINED_S:
+        return tfl_sustained, "tensor", "bf16_tflops_sustained"
+    return tfl_burst, "tensor", "bf16_tflops"
+
+
 def _workload(name, page_size=16):
     from paged_kv_cache_376_b200 import workloads as W
     if name == "tiny":
@@ -544,14 +556,7 @@ def run_tv(args, rank, world, local_rank):
                    "balanced": "tv_paged_decode_balanced"}[runner.kind]
     if runner.engine:
         kernel_name = "tv_decode_step"
-    if unit == "GB/s":
-        peak, bound, key = hbm, "hbm", "hbm_gbs"
-    elif wall >= SUSTAINED_S:
-        # a timed region of seconds runs under the 1 kW power cap: the
-        # GEMM figure measured the same way; shorter ones are bursts
-        peak, bound, key = tfl_sus, "tensor", "bf16_tflops_sustained"
-    else:
-        peak, bound, key = tfl, "tensor", "bf16_tflops"
+    peak, bound, key = _roofline_peak(unit, wall, hbm, tfl, tfl_sus)
     res = {
         "metric": METRIC if args.workload != "prefill" else
         "chunked prefill causal attention TFLOP/s (% of B200 bf16 peak)",

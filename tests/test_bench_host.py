@@ -129,3 +129,16 @@ def test_cpu_baseline_reports_all_cores_and_one_core():
     one = r["single_core"]
     assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == "GB/s"
     assert oracle.max_threads() == cores        # thread count restored
+
+
+def test_roofline_peak_follows_the_bound_and_the_timed_region():
+    hbm, burst, sus = 6538.3, 1637.9, 1372.1
+    assert bench._roofline_peak("GB/s", 0.01, hbm, burst, sus) == \
+        (hbm, "hbm", "hbm_gbs")
+    assert bench._roofline_peak("GB/s", 30.0, hbm, burst, sus) == \
+        (hbm, "hbm", "hbm_gbs")
+    assert bench._roofline_peak("TFLOP/s", 0.006, hbm, burst, sus) == \
+        (burst, "tensor", "bf16_tflops")
+    assert bench._roofline_peak("TFLOP/s", bench.SUSTAINED_S, hbm, burst,
+                                sus) == (sus, "tensor",
+                                         "bf16_tflops_sustained")
