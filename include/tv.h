@@ -35,9 +35,9 @@
  *   - Query head h reads KV head h / (num_q_heads / num_kv_heads).
  *   - Supported: head_dim == 64, page_size 16 or 32 ([P3] recommends 16-32
  *     tokens; the kernels stream 16-token blocks, two per 32-token page),
- *     num_q_heads a multiple of
- *     num_kv_heads with a ratio in {1, 2, 4, 8}; every pointer 16-byte
- *     aligned; num_seqs <= 65535; num_pages * page_size and
+ *     num_q_heads a multiple of num_kv_heads with a ratio in {1, 2, 4, 8}
+ *     (tv_paged_prefill: 4 only); every pointer 16-byte aligned; num_seqs
+ *     <= 65535; num_pages * page_size and
  *     max_blocks_per_seq * page_size at most INT32_MAX (token positions and
  *     pool rows are 32-bit in the kernels).  Anything else returns
  *     TV_ERR_UNSUPPORTED or TV_ERR_INVALID_ARG before any launch.
@@ -281,6 +281,10 @@ tv_status tv_split_merge(void* out, const float* partial_out,
  *                    separate workspaces.
  *   workspace_bytes  its size
  * A sequence with T_s > C is flagged TV_DEVERR_BAD_QUERY and skipped.
+ * Supported: num_q_heads == 4 * num_kv_heads (TV_ERR_UNSUPPORTED
+ * otherwise) and scale > 0 (TV_ERR_INVALID_ARG otherwise: the kernel takes
+ * each key tile's maximum on the raw scores q.K and scales it afterwards,
+ * which equals the maximum of the scaled scores only for a positive scale).
  */
 tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
                            const int32_t* query_start_loc, const void* k_pool,
@@ -323,6 +327,11 @@ tv_status tv_prefill_workspace_size(int num_seqs, int max_query_len,
  *     streams) race on it;
  *   - the first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept per device together with the id of the CUDA
+ *     context it belongs to; when a later call finds another context
+ *     current (e.g. after cudaDeviceReset) it looks the address up again,
+ *     so that first call in the new context should also come before any
+ *     capture.
  * Returns TV_ERR_CUDA when that lookup fails.
  */
 #define TV_STATIC_SCRATCH_FLOATS (1 << 23)
@@ -364,13 +373,20 @@ tv_status tv_selftest_wait_timeout(uint32_t* err, int64_t limit_ns,
  * caller-owned, set up by tv_pool_init and changed only by the tv_pool_*
  * calls:
  *   [0] number of free pages (top of the stack)   [2] slots written by the
- *   last tv_pool_append_slots   [3] page size   [4 .. 4+NP) free-page stack (pop takes entry
- *   top-1)   then NP reference counts and 2 x NP scratch words.
+ *   last tv_pool_append_slots   [3] page size   [4 .. 4+NP) free-page stack
+ *   (pop takes entry top-1)   then NP reference counts, 2 x NP scratch
+ *   words (zero between calls) and TV_POOL_MAX_SEQS growth marks: entry s
+ *   is 1 when the last tv_pool_append_slots gave sequence s its tokens, 0
+ *   when it did not (no tokens asked, pool exhausted, or a flagged error);
+ *   entries at and beyond that call's num_seqs are left as they were.
  * A page's reference count is the number of block-table rows holding it.
- * Every pool call serves at most 1024 sequences (TV_ERR_UNSUPPORTED above),
- * runs as one CTA, and is ordered with the caller's other work by `stream`.
+ * Every pool call serves at most TV_POOL_MAX_SEQS sequences
+ * (TV_ERR_UNSUPPORTED above), runs as one CTA, and is ordered with the
+ * caller's other work by `stream`.
  */
-#define TV_POOL_STATE_INTS(num_pages) (4 + 4 * (int64_t)(num_pages))
+#define TV_POOL_MAX_SEQS 1024
+#define TV_POOL_STATE_INTS(num_pages) \
+  (4 + 4 * (int64_t)(num_pages) + TV_POOL_MAX_SEQS)
 
 /*
  * tv_pool_init -- every page free, except those the first
@@ -446,13 +462,16 @@ tv_status tv_pool_release(int32_t* pool_state, int64_t num_pages,
  * tv_paged_decode_append (the new token's K/V go to position ctx-1 of the
  * grown context; out = attention of q over it), or, when workspace is not
  * NULL, tv_paged_decode_balanced with k_new / v_new and that workspace (for
- * batches of mixed lengths).  Sequences with context 0
- * are idle: they append nothing and output zeros.  Two launches, no host
- * synchronisation, so a run of steps can be captured in one CUDA graph.
- * A sequence left unserved by an empty pool (TV_DEVERR_POOL_EMPTY) has its
- * last cached row overwritten by this step's row: keep at least one free
- * page per live sequence.  Arguments as tv_pool_append_slots and
- * tv_paged_decode_append.
+ * batches of mixed lengths).  Only the sequences whose context the slot
+ * reservation grew (growth mark 1 in pool_state) append and attend; every
+ * other sequence is idle for this step: it appends nothing, its output row
+ * is zeros and its pages are left untouched.  That covers context 0, a
+ * sequence left unserved by an exhausted pool (TV_DEVERR_POOL_EMPTY; it
+ * keeps its context and every cached row, and can be stepped again once
+ * pages are released) and one flagged TV_DEVERR_BAD_CONTEXT (full) or
+ * TV_DEVERR_BAD_PAGE.  Two launches, no host synchronisation, so a run of
+ * steps can be captured in one CUDA graph.  Arguments as
+ * tv_pool_append_slots and tv_paged_decode_append.
  */
 tv_status tv_decode_step(int32_t* pool_state, int64_t num_pages, void* out,
                          const void* q, const void* k_new, const void* v_new,

@@ -377,9 +377,12 @@ def tv_paged_decode_balanced(out, q, k_pool, v_pool, block_tables,
 
 # ---- device page pool --------------------------------------------------------
 
+POOL_MAX_SEQS = 1024   # TV_POOL_MAX_SEQS
+
+
 def pool_state_ints(num_pages):
     """TV_POOL_STATE_INTS(num_pages) of include/tv.h."""
-    return 4 + 4 * int(num_pages)
+    return 4 + 4 * int(num_pages) + POOL_MAX_SEQS
 
 
 def pool_state(num_pages, device=None):
@@ -398,9 +401,10 @@ def _pool_tables(block_tables, context_lens):
 
 def _pool_pages(state):
     _cuda(state, torch.int32, "pool_state")
-    n = state.numel() - 4
+    n = state.numel() - 4 - POOL_MAX_SEQS
     if n <= 0 or n % 4:
-        raise ValueError("pool_state must hold 4 + 4 * num_pages ints")
+        raise ValueError("pool_state must hold TV_POOL_STATE_INTS(num_pages)"
+                         " = 4 + 4 * num_pages + 1024 ints")
     return n // 4
 
 

@@ -43,6 +43,8 @@ struct PoolView {
   int32_t* ref;          // [num_pages]
   int32_t* cnt_app;      // [num_pages], zero between calls
   int32_t* last_app;     // [num_pages], zero between calls
+  int32_t* grown;        // [kPoolMaxSeqs]: 1 = got its tokens in the last
+                         // append call, 0 = did not (idle, unserved, flagged)
   int num_pages;
 };
 
@@ -55,6 +57,7 @@ __host__ __device__ inline PoolView view(int32_t* state, int num_pages) {
   v.ref = v.stack + num_pages;
   v.cnt_app = v.ref + num_pages;
   v.last_app = v.cnt_app + num_pages;
+  v.grown = v.last_app + num_pages;
   v.num_pages = num_pages;
   return v;
 }
@@ -101,6 +104,9 @@ __global__ void pool_clear_kernel(PoolView p) {
     p.cnt_app[i] = 0;
     p.last_app[i] = 0;
   }
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kPoolMaxSeqs;
+       i += gridDim.x * blockDim.x)
+    p.grown[i] = 0;
 }
 
 __global__ void pool_count_refs_kernel(PoolView p, const int32_t* bt, int mb,
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int job_old[kThreads], job_new[kThreads];
   if (*p.page_size != kPS) {   // pools of another page size: touch nothing
     if (threadIdx.x == 0) flag_error(err, DEVERR_BAD_SEQ);
+    if (threadIdx.x < num_seqs) p.grown[threadIdx.x] = 0;
     return;
   }
   const int s = threadIdx.x;
@@ -198,6 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int off = block_exclusive_scan(need, sh, &total);
   const bool served = live && n > 0 && off + need <= top;
   if (live && n > 0 && !served) flag_error(err, DEVERR_POOL_EMPTY);
+  // what a decode step launched next reads: only a sequence whose context
+  // grew may append at its last position (any other would overwrite a
+  // cached token there)
+  if (live) p.grown[s] = served ? 1 : 0;
   int used;
   const int served_need = served ? need : 0;
   (void)block_exclusive_scan(served_need, sh, &used);

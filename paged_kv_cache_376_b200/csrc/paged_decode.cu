@@ -81,7 +81,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int chk = lane & 7;    // 16-byte chunk of the head dim
 
   // ---- token range of this CTA --------------------------------------------
-  int ctx = a.context_lens[seq];
+  // a decode step (tv_decode_step) treats a sequence whose context did not
+  // grow as idle: appending at ctx-1 would overwrite a cached token
+  int ctx = (a.grown && a.grown[seq] == 0) ? 0 : a.context_lens[seq];
   // A page holds 1 << page_shift blocks of 16 tokens; the kernel streams
   // blocks, and a block's 16 rows are one TMA box at row (page << shift |
   // sub-block) * 16 of the pool.

@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
   // ---- pages per sequence, exclusive prefix in shared memory ---------------
   for (int s = threadIdx.x; s < B; s += kThreads) {
-    const int raw = a.context_lens[s];
+    // in a decode step, a sequence whose context did not grow is idle
+    const int raw = (a.grown && a.grown[s] == 0) ? 0 : a.context_lens[s];
     if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0)
       flag_error(a.err, DEVERR_BAD_CONTEXT);
     const int ctx = clamp_ctx(raw, ctx_cap);

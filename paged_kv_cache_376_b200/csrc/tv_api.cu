@@ -203,7 +203,8 @@ static tv_status decode_common(void* out, float* partial_out,
                                int page_size, int64_t num_pages, float scale,
                                int partition_tokens, int max_partitions,
                                bool split, uint32_t* err, void* stream,
-                               const BalancedWorkspace* ws = nullptr) {
+                               const BalancedWorkspace* ws = nullptr,
+                               const int32_t* grown = nullptr) {
   tv_status st =
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
   if (st != TV_OK) return st;
@@ -257,6 +258,7 @@ static tv_status decode_common(void* out, float* partial_out,
   a.v_pool_w = static_cast<__nv_bfloat16*>(const_cast<void*>(v_pool));
   a.block_tables = block_tables;
   a.context_lens = context_lens;
+  a.grown = grown;
   a.err = err;
   a.max_blocks_per_seq = max_blocks_per_seq;
   a.num_q_heads = num_q_heads;
@@ -381,7 +383,7 @@ static tv_status pool_common(const int32_t* pool_state, int64_t num_pages,
       (num_seqs > 0 &&
        (!block_tables || !context_lens || max_blocks_per_seq <= 0)))
     return TV_ERR_INVALID_ARG;
-  if (num_pages > (INT32_MAX - 4) / 4 || num_seqs > tv::kPoolMaxSeqs ||
+  if (num_pages > (INT32_MAX - 4) / 4 || num_seqs > TV_POOL_MAX_SEQS ||
       (int64_t)max_blocks_per_seq * 32 > INT32_MAX)
     return TV_ERR_UNSUPPORTED;
   return TV_OK;
@@ -479,17 +481,17 @@ tv_status tv_decode_step(int32_t* pool_state, int64_t num_pages, void* out,
                             num_seqs, nullptr, k_pool, v_pool, num_kv_heads,
                             head_dim, page_size, err, stream);
   if (st != TV_OK) return st;
-  if (workspace)
-    return tv_paged_decode_balanced(
-        out, q, k_new, v_new, k_pool, v_pool, block_tables,
-        max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
-        head_dim, page_size, num_pages, scale, workspace, workspace_bytes, err,
-        stream);
-  return tv_paged_decode_append(out, q, k_new, v_new, k_pool, v_pool,
-                                block_tables, max_blocks_per_seq,
-                                context_lens, num_seqs, num_q_heads,
-                                num_kv_heads, head_dim, page_size, num_pages,
-                                scale, err, stream);
+  if (num_seqs == 0) return TV_OK;
+  // the pool's marks of the sequences that got room for their token: every
+  // other sequence is idle in the attention launch (appends nothing, zero
+  // output), so a sequence left unserved keeps its cached rows intact
+  const int32_t* grown = pool_state + 4 + 4 * num_pages;
+  const BalancedWorkspace ws{workspace, workspace_bytes};
+  return decode_common(out, nullptr, nullptr, q, k_new, v_new, k_pool, v_pool,
+                       block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, 0, 1, false, err, stream,
+                       workspace ? &ws : nullptr, grown);
 }
 
 tv_status tv_paged_decode_split(float* partial_out, float* partial_lse,
@@ -555,8 +557,11 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
   if (st != TV_OK) return st;
   if (num_q_heads / num_kv_heads != 4) return TV_ERR_UNSUPPORTED;
+  // the kernel scales each tile's maximum raw score, which is the maximum
+  // of the scaled scores only when the scale is positive
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
-      max_query_len < 0 || num_query_rows < 0 || !std::isfinite(scale))
+      max_query_len < 0 || num_query_rows < 0 || !std::isfinite(scale) ||
+      !(scale > 0.f))
     return TV_ERR_INVALID_ARG;
   if (num_seqs > 65535 || num_pages * page_size > INT32_MAX ||
       (int64_t)max_blocks_per_seq * page_size > INT32_MAX)

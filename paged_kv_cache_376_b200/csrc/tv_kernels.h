@@ -19,6 +19,10 @@ struct DecodeArgs {
   __nv_bfloat16* v_pool_w;
   const int32_t* block_tables;   // [B][max_blocks_per_seq]
   const int32_t* context_lens;   // [B]
+  // nullable; grown[s] == 0 makes sequence s idle (no append, zero output):
+  // the pool's marks of the sequences whose context the step's slot
+  // reservation grew (tv_decode_step only)
+  const int32_t* grown;
   uint32_t* err;                 // nullable
   int max_blocks_per_seq;
   int num_q_heads;

@@ -25,11 +25,17 @@
 //     events;
 //   * the first call on a device looks up the array's device address with
 //     that device current (cudaGetSymbolAddress); make that first call before
-//     any stream capture.
+//     any stream capture.  The address is remembered together with the
+//     identity of the CUDA context it was looked up in; a call that finds
+//     another context current (after cudaDeviceReset the runtime makes a new
+//     primary context, which loads the library's kernels and the array
+//     afresh) looks it up again instead of using an address of the old one.
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "tv.h"
 
@@ -43,19 +49,56 @@ static __device__ __align__(256) float g_tv_split_scratch[TV_STATIC_SCRATCH_FLOA
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};   // context id, 0 = none
 
-// Device address of the scratch on the current device, looked up once per
-// device with that device current.  nullptr on failure.
+// Unique id of the CUDA context current on this thread (ids are never
+// reused within a process), or 0 when none is current or it cannot be read.
+// The driver calls come through the runtime's entry-point lookup, so the
+// library needs no link against libcuda.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch on the current device, looked up with that
+// device current the first time it is used in the current context (normally
+// once per device).  nullptr on failure.
 float* scratch_on_current_device() {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_tv_split_scratch);
-    if (e != cudaSuccess || p == nullptr) return nullptr;
+    if (e != cudaSuccess || p == nullptr) {
+      g_scratch_ptr[dev] = nullptr;
+      return nullptr;
+    }
     g_scratch_ptr[dev] = static_cast<float*>(p);
+    // the lookup makes the device's primary context current if none was
+    g_scratch_ctx[dev] = current_context_id();
   }
   return g_scratch_ptr[dev];
 }

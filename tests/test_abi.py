@@ -97,6 +97,30 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
                                 None) == 1
 
 
+def test_prefill_refuses_a_scale_that_is_not_positive(lib):
+    """The prefill kernel scales each key tile's maximum raw score; that is
+    the maximum of the scaled scores only for scale > 0, so anything else is
+    refused instead of silently overflowing the exponentials."""
+    p = _fake()
+    for scale in (-0.125, 0.0, -0.0, float("-inf")):
+        assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, 4, p, 1, 8, 32, 8,
+                                    64, 16, 10, scale, None, 0, None,
+                                    None) == 1, scale
+
+
+def test_pool_state_size_includes_the_growth_marks(lib):
+    """TV_POOL_STATE_INTS(np) = 4 + 4 np + TV_POOL_MAX_SEQS (include/tv.h);
+    the binding sizes and checks state arrays by the same rule."""
+    hdr = open(os.path.join(ROOT, "include", "tv.h")).read()
+    assert re.search(r"#define TV_POOL_MAX_SEQS 1024\b", hdr)
+    assert _lib.POOL_MAX_SEQS == 1024
+    assert _lib.pool_state_ints(10) == 4 + 40 + 1024
+    # more sequences than the marks cover are refused before any launch
+    p = _fake()
+    assert lib.tv_pool_append_slots(p, 10, p, 4, p, None, 1025, None, p, p,
+                                    8, 64, 16, None, None) == 2
+
+
 def test_sizes_beyond_32_bit_positions_are_refused(lib):
     p = _fake()
     big_mb = 1 << 27          # x 16-token pages = 2^31 token positions

@@ -54,6 +54,8 @@ class Both:
         self.g_kp = _bits(kp.view(np.int16))
         self.g_vp = _bits(vp.view(np.int16))
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        # growth marks: 1 where the last append call gave a sequence tokens
+        self.grown = np.zeros(batch, np.int32)
         _lib.tv_pool_init(self.g_state, err=self.err)
 
     def check(self):
@@ -67,7 +69,9 @@ class Both:
         n = self.np_
         np.testing.assert_array_equal(st[4 + n:4 + 2 * n], self.pool.ref)
         # the scratch words are back at zero
-        assert not st[4 + 2 * n:].any()
+        assert not st[4 + 2 * n:4 + 4 * n].any()
+        np.testing.assert_array_equal(st[4 + 4 * n:4 + 4 * n + self.b],
+                                      self.grown)
         np.testing.assert_array_equal(bf16_bits(self.g_kp), self.kp)
         np.testing.assert_array_equal(bf16_bits(self.g_vp), self.vp)
 
@@ -82,6 +86,7 @@ class Both:
                                   num_new_tokens=_i32(n_new),
                                   slot_mapping=g_slots, err=self.err)
         torch.cuda.synchronize()
+        self.grown = (served & (np.asarray(n_new) > 0)).astype(np.int32)
         assert int(self.g_state[2]) == len(slots)
         np.testing.assert_array_equal(g_slots[:len(slots)].cpu().numpy(),
                                       slots)
@@ -276,3 +281,105 @@ def test_graph_captured_decode_steps_match_the_oracle(balanced):
         np.testing.assert_array_equal(bf16_bits(g["vp"]), vp)
         assert_parity(g["out"], ref, f"decode step {step}")
     assert int(err.item()) == 0
+
+
+@pytest.mark.parametrize("balanced", [False, True],
+                         ids=["per-pair", "balanced"])
+def test_exhausted_pool_leaves_unserved_sequences_untouched(balanced):
+    """An exhausted pool inside graph-replayed decode steps: a sequence that
+    gets no room for its token (and every later one in batch order) is idle
+    for the step -- its cached rows, its context and the pages it shares
+    with a fork stay bit for bit as they were, and its output row is zero --
+    while the served ones append and attend as the oracle says.  Pages are
+    released between steps until everyone is served again.
+
+    Sequences (batch order): A (16 cached tokens: its next token opens a
+    page), B = fork of A, D (20 cached: its next token goes into a partly
+    filled page that E shares, so D must copy it first), E = fork of D.  The
+    pool has one free page."""
+    batch, mb = 4, 8
+    # the workload caches 16 and 20 tokens of A and D (its own append slot
+    # at position 16 / 20 is not used here)
+    wl = W.decode_workload([17, 21], num_pages=4, seed=31)
+    bt = np.full((batch, mb), -1, np.int64)
+    ctx = np.zeros(batch, np.int64)
+    bt[0, :1] = wl.block_tables[0, :1]
+    bt[2, :2] = wl.block_tables[1, :2]
+    ctx[0], ctx[2] = 16, 20
+    kp, vp = wl.k_pool.copy(), wl.v_pool.copy()
+    pool = PagePool(wl.num_pages, bt, ctx)
+    assert pool.top == 1
+    g = dict(bt=_i32(bt), ctx=_i32(ctx), kp=_bits(kp.view(np.int16)),
+             vp=_bits(vp.view(np.int16)),
+             q=torch.empty((batch, 32, D), dtype=torch.bfloat16, device="cuda"),
+             kn=torch.empty((batch, HKV, D), dtype=torch.bfloat16,
+                            device="cuda"),
+             vn=torch.empty((batch, HKV, D), dtype=torch.bfloat16,
+                            device="cuda"),
+             out=torch.empty((batch, 32, D), dtype=torch.bfloat16,
+                             device="cuda"))
+    st = _lib.pool_state(wl.num_pages)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _lib.tv_pool_init(st, g["bt"], g["ctx"])
+    pool.fork(bt, ctx, [(0, 1), (2, 3)])
+    _lib.tv_pool_fork(st, g["bt"], g["ctx"], _i32([0, 2]), _i32([1, 3]))
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    ws = _lib.decode_workspace(batch, 32, HKV) if balanced else None
+    with torch.cuda.graph(graph, stream=side):
+        _lib.tv_decode_step(st, g["out"], g["q"], g["kn"], g["vn"], g["kp"],
+                            g["vp"], g["bt"], g["ctx"], wl.scale,
+                            workspace=ws, err=err)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(32)
+
+    def draw(shape):
+        return W.bf16_bits(rng.standard_normal(shape).astype(np.float32))
+
+    # (sequences released before the step, sequences served by the step)
+    plan = [([], [0]), ([0], [1]), ([1], [2, 3]), ([], [2, 3])]
+    for step, (release, want_served) in enumerate(plan):
+        if release:
+            pool.release(bt, ctx, release)
+            _lib.tv_pool_release(st, g["bt"], g["ctx"], _i32(release))
+        q, kn, vn = draw((batch, 32, D)), draw((batch, HKV, D)), \
+            draw((batch, HKV, D))
+        g["q"].copy_(_bits(q.view(np.int16)))
+        g["kn"].copy_(_bits(kn.view(np.int16)))
+        g["vn"].copy_(_bits(vn.view(np.int16)))
+        g["out"].fill_(float("nan"))
+        err.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        live = (ctx > 0).astype(np.int64)
+        before = ctx.copy()
+        _, served = pool.append_slots(bt, ctx, live, kp, vp)
+        grown = served & (live > 0)
+        assert np.flatnonzero(grown).tolist() == want_served, step
+        sl = np.full(batch, -1, np.int32)
+        for s in np.flatnonzero(grown):
+            t = ctx[s] - 1
+            sl[s] = bt[s][t // PAGE] * PAGE + t % PAGE
+        kp, vp, bad = oracle.kv_append(kn, vn, sl, kp, vp)
+        assert bad == 0
+        att_ctx = np.where(grown, ctx, 0).astype(np.int32)
+        ref = oracle.paged_decode(q, kp, vp, bt.astype(np.int32), att_ctx,
+                                  wl.scale)
+        np.testing.assert_array_equal(g["bt"].cpu().numpy(), bt)
+        np.testing.assert_array_equal(g["ctx"].cpu().numpy(), ctx)
+        # cached rows of every sequence, shared pages included, bit-exact
+        np.testing.assert_array_equal(bf16_bits(g["kp"]), kp)
+        np.testing.assert_array_equal(bf16_bits(g["vp"]), vp)
+        n = wl.num_pages
+        np.testing.assert_array_equal(
+            st.cpu().numpy()[4 + 4 * n:4 + 4 * n + batch], grown)
+        out = g["out"].cpu().float().numpy()
+        for s in range(batch):
+            if not grown[s]:
+                assert (out[s] == 0).all(), (step, s)
+        assert_parity(g["out"][torch.tensor(grown, device="cuda")],
+                      ref[grown], f"served rows, step {step}")
+        want_err = _lib.DEVERR_POOL_EMPTY if step < 2 else 0
+        assert int(err.item()) == want_err, step

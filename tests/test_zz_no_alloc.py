@@ -5,7 +5,9 @@ nearly all device memory to the KV page pool, step loops that cannot afford
 cudaMalloc's blocking, C hosts without a device allocator).  Its output must
 match the existing two-call path (tv_paged_decode_split into caller buffers,
 then tv_split_merge) within the parity bound of the other tests, on two calls
-in a row, since every call reuses the same library-owned scratch array.
+in a row, since every call reuses the same library-owned scratch array; and,
+because both paths run the same kernels, it must also match the fp64 CPU
+oracle's decode directly, so that a fault the two share cannot hide.
 
 This file is collected last so that, if it fails, a run stopping at the first
 failure has already run every other test.
@@ -15,8 +17,10 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from gpu_util import (REL, ABS, assert_parity, err_word, gpu_append,
-                      gpu_merge, gpu_split, require_gpu, to_f64, upload)
+                      gpu_merge, gpu_split, oracle_after_append, require_gpu,
+                      to_f64, upload)
 from paged_kv_cache_376_b200 import _lib
 from paged_kv_cache_376_b200 import workloads as W
 
@@ -56,6 +60,11 @@ def test_static_scratch_matches_the_two_call_path_on_consecutive_calls():
         torch.cuda.synchronize()
         assert_parity(got, to_f64(want), f"static scratch, batch {wl.num_seqs}",
                       rel=REL, abs_=ABS)
+        kp, vp = oracle_after_append(wl)
+        ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables,
+                                  wl.context_lens, wl.scale)
+        assert_parity(got, ref, f"static scratch vs oracle, batch "
+                      f"{wl.num_seqs}", rel=REL, abs_=ABS)
         assert err_word(db) == 0
 
 
