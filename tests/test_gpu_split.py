@@ -87,12 +87,16 @@ def test_one_partition_equals_unsplit_decode_bitwise():
     np.testing.assert_array_equal(bf16_bits(merged), bf16_bits(direct))
 
 
-def test_long_split_config_sampled_rows_and_needles():
+def test_long_split_config_every_row_partials_and_needles():
+    """The 8 x 131072-token configuration at full size, in the launch shape
+    the benchmark times (512-token partitions): every (sequence, head) output
+    row and every partial (o_p, lse_p) against the oracle, plus planted
+    needles whose output must equal their V row bit for bit."""
     wl = W.long_split()
     pt = wl.partition_tokens
     maxp = wl.max_partitions()
     kp, vp = oracle_after_append(wl)
-    # needles: sequence 1 head group 2 at the first, a middle and the last
+    # needles: sequence s, head group 2, at the first, a middle and the last
     # partition, and at a page's last slot; each needle query group shares q
     q = wl.q.copy()
     needles = {1: 5, 3: 131072 // 2 + 77, 5: 131071 - 3, 6: 16 * 4000 + 15}
@@ -108,16 +112,15 @@ def test_long_split_config_sampled_rows_and_needles():
     out = gpu_merge(db, po, pl, pt)
     torch.cuda.synchronize()
     assert err_word(db) == 0
-    rng = np.random.default_rng(4)
-    si = rng.integers(0, wl.num_seqs, 12).astype(np.int32)
-    hi = rng.integers(0, wl.num_q_heads, 12).astype(np.int32)
-    ref = oracle.paged_decode_rows(wl.q, kp, vp, wl.block_tables,
-                                   wl.context_lens, wl.scale, si, hi)
-    assert_parity(out[torch.from_numpy(si).long(),
-                      torch.from_numpy(hi).long()], ref, "long sampled")
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, "long, every row")
+    ro, rl = oracle.paged_decode_partials(wl.q, kp, vp, wl.block_tables,
+                                          wl.context_lens, wl.scale, pt, maxp)
+    assert_parity(po, ro, "long, every o_p")
+    _lse_close(pl, rl, "long, every lse_p")
     for s, pos in needles.items():
         page, off = wl.block_tables[s, pos // 16], pos % 16
         got = bf16_bits(out[s, 8:12])
         np.testing.assert_array_equal(got, np.repeat(vp[page, off, 2][None],
                                                      4, axis=0))
-    assert torch.isfinite(out.float()).all()
