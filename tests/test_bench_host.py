@@ -150,3 +150,22 @@ def test_roofline_peak_follows_the_bound_and_the_timed_region():
     assert bench._roofline_peak("TFLOP/s", bench.SUSTAINED_S, hbm, burst,
                                 sus) == (sus, "tensor",
                                          "bf16_tflops_sustained")
+
+
+def test_l2_is_flushed_only_where_the_working_set_could_stay_in_l2():
+    """Steps whose touched bytes (cached K/V + q + out) are under twice the
+    126 MB L2 are timed one by one with L2 flushed in between; the decode
+    configurations stream more than that and run back to back."""
+    tiny = W.tiny_decode()
+    assert bench.working_set_bytes(tiny) == (tiny.kv_bytes_read()
+                                             + 2 * tiny.q.nbytes)
+    assert bench.flushes_l2(tiny)
+    small_prefill = W.prefill_workload([100, 0], [64, 64], seed=3)
+    assert bench.flushes_l2(small_prefill)
+    # 64 x 2048 tokens x 2 KB = 268 MB of K/V: more than twice L2
+    big = W.decode_workload([2048] * 64, num_pages=8192, seed=4)
+    assert big.kv_bytes_read() == 268435456
+    assert not bench.flushes_l2(big)
+    assert bench.flushes_l2(big, l2_bytes=1 << 30)
+    cfg = bench._config(tiny, "tiny")
+    assert "flushed" in cfg["l2"]
