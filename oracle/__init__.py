@@ -31,7 +31,9 @@ def build(force: bool = False) -> str:
             and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+    # binary32 steps stay unfused (the RoPE reading fixes each rounding)
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp",
+           "-fPIC", "-shared",
            "-o", tmp, _SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, _LIB_PATH)
@@ -63,6 +65,8 @@ def _load():
     lib.oracle_paged_prefill_rows.argtypes = [
         P, P, P, i64, P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, dbl]
     lib.oracle_paged_prefill_rows.restype = i64
+    lib.oracle_rope_rows.argtypes = [P, P, i64, i32, i32, P, i32]
+    lib.oracle_rope_rows.restype = i64
     _lib = lib
     return lib
 
@@ -98,6 +102,33 @@ def kv_append(k_new, v_new, slot_mapping, k_pool, v_pool):
                                _ptr(kp), _ptr(vp), num_pages, hkv, d,
                                page_size)
     return kp, vp, int(bad)
+
+
+def rope(rows, positions, cos_sin):
+    """RoPE of K rows (oracle.c: oracle_rope_rows): a rotated copy of the
+    uint16 bf16 rows [T][num_kv_heads][head_dim] at the given positions, with
+    angles from cos_sin float32 [max_position][2][head_dim // 2] (cos row,
+    then sin row).  Also returns the count of rows whose position is outside
+    the table (left unrotated)."""
+    lib = _load()
+    out = np.array(rows, dtype=np.uint16, copy=True, order="C")
+    pos = _c(positions, np.int32)
+    cs = _c(cos_sin, np.float32)
+    t, hkv, d = out.shape
+    if cs.ndim != 3 or cs.shape[1:] != (2, d // 2):
+        raise ValueError("cos_sin must be [max_position][2][head_dim // 2]")
+    bad = lib.oracle_rope_rows(_ptr(out), _ptr(pos), t, hkv, d, _ptr(cs),
+                               cs.shape[0])
+    return out, int(bad)
+
+
+def kv_append_rope(k_new, v_new, slot_mapping, positions, cos_sin, k_pool,
+                   v_pool):
+    """kv_append with each new K row rotated at its position first (V is not
+    rotated)."""
+    k_rot, bad_pos = rope(k_new, positions, cos_sin)
+    kp, vp, bad = kv_append(k_rot, v_new, slot_mapping, k_pool, v_pool)
+    return kp, vp, bad, bad_pos
 
 
 def paged_decode_rows(q, k_pool, v_pool, block_tables, context_lens, scale,

@@ -139,6 +139,62 @@ static int attend(const uint16_t *q, const uint16_t *k_pool,
     return bad;
 }
 
+/*
+ * RoPE on K rows ([P1] sec. "Llama 3.2 1B架构拆解": rotary position encoding
+ * injects the position into Q and K by rotation).  The pages give neither
+ * the pairing of dimensions nor the angles nor the arithmetic; the readings:
+ *   - dimension i is rotated together with i + head_dim/2 (the rotate-half
+ *     convention of the Hugging Face Llama model the pages dump);
+ *   - the angles come from a caller table cos_sin[position][2][head_dim/2]
+ *     (the cos row, then the sin row), so any frequency base or scaling is
+ *     the caller's;
+ *   - the arithmetic is binary32: with x1 = k[i], x2 = k[i + D/2],
+ *       y1 = fl(fl(x1 * c) - fl(x2 * s)),  y2 = fl(fl(x2 * c) + fl(x1 * s)),
+ *     fl() rounding to nearest binary32 (no fused multiply-add), and the
+ *     result is rounded to bf16 (nearest even) as it enters the pool.
+ * A row whose position is outside [0, max_position) is left unrotated and
+ * counted.
+ */
+static uint16_t bf16_round_nearest_even(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return (uint16_t)((u >> 16) | 0x40u);          /* quiet NaN */
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+int64_t oracle_rope_rows(uint16_t *rows, const int32_t *positions,
+                         int64_t num_rows, int num_kv_heads, int head_dim,
+                         const float *cos_sin, int max_position)
+{
+    const int half = head_dim / 2;
+    int64_t bad = 0;
+    for (int64_t t = 0; t < num_rows; ++t) {
+        const int pos = positions[t];
+        if (pos < 0 || pos >= max_position) {
+            ++bad;
+            continue;
+        }
+        const float *cs = cos_sin + (int64_t)pos * head_dim;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            uint16_t *k = rows + (t * num_kv_heads + h) * (int64_t)head_dim;
+            for (int i = 0; i < half; ++i) {
+                const float x1 = (float)bf16_value(k[i]);
+                const float x2 = (float)bf16_value(k[i + half]);
+                const float c = cs[i], s = cs[half + i];
+                const float a = x1 * c, b = x2 * s;
+                const float e = x2 * c, f = x1 * s;
+                const float y1 = a - b, y2 = e + f;
+                k[i] = bf16_round_nearest_even(y1);
+                k[i + half] = bf16_round_nearest_even(y2);
+            }
+        }
+    }
+    return bad;
+}
+
 void oracle_set_threads(int n)
 {
 #ifdef _OPENMP

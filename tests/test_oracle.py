@@ -372,3 +372,122 @@ def test_workload_append_fills_the_last_position():
         np.testing.assert_array_equal(kp[page, pos % 16], wl.k_new[s])
         # the append landed in a page already holding earlier tokens
         assert not np.isnan(W.bf16_to_f64(wl.k_pool[page, 0])).any()
+
+
+
+# ---- RoPE on K (oracle.rope) ---------------------------------------------------
+
+def _rope_table(angles):
+    """cos_sin [positions][2][half] float32 from fp64 angles [positions][half]."""
+    a = np.asarray(angles, dtype=np.float64)
+    return np.stack([np.cos(a), np.sin(a)], axis=1).astype(np.float32)
+
+
+def _bf16_rows(rng, shape):
+    return W.bf16_bits(rng.standard_normal(shape).astype(np.float32))
+
+
+def test_rope_golden_pairs_worked_by_hand():
+    path = os.path.join(os.path.dirname(__file__), "golden", "rope_example.txt")
+    for line in open(path):
+        line = line.split("#")[0].split()
+        if not line:
+            continue
+        x1, x2, c, s, y1, y2 = line
+        d = 64
+        rows = np.zeros((1, 1, d), np.uint16)
+        rows[0, 0, 5], rows[0, 0, 5 + d // 2] = int(x1, 16), int(x2, 16)
+        cs = np.zeros((1, 2, d // 2), np.float32)
+        cs[0, 0, :], cs[0, 1, :] = 1.0, 0.0
+        cs[0, 0, 5], cs[0, 1, 5] = float(c), float(s)
+        out, bad = oracle.rope(rows, np.array([0], np.int32), cs)
+        assert bad == 0
+        assert (int(out[0, 0, 5]), int(out[0, 0, 5 + d // 2])) == \
+            (int(y1, 16), int(y2, 16))
+        # every other pair sees angle 0: unchanged
+        keep = np.ones(d, bool)
+        keep[[5, 5 + d // 2]] = False
+        np.testing.assert_array_equal(out[0, 0, keep], rows[0, 0, keep])
+
+
+def test_rope_exact_turns():
+    rng = np.random.default_rng(61)
+    rows = _bf16_rows(rng, (5, 8, 64))
+    pos = np.arange(5, dtype=np.int32)
+    # 0, a quarter, half and three quarters of a turn, for every pair
+    cs = np.zeros((5, 2, 32), np.float32)
+    cs[0, 0], cs[0, 1] = 1, 0
+    cs[1, 0], cs[1, 1] = 0, 1
+    cs[2, 0], cs[2, 1] = -1, 0
+    cs[3, 0], cs[3, 1] = 0, -1
+    cs[4, 0], cs[4, 1] = 1, 0
+    out, bad = oracle.rope(rows, pos, cs)
+    assert bad == 0
+    x1, x2 = rows[..., :32], rows[..., 32:]
+    neg = lambda b: b ^ np.uint16(0x8000)
+    np.testing.assert_array_equal(out[0], rows[0])
+    np.testing.assert_array_equal(out[1, :, :32], neg(x2[1]))
+    np.testing.assert_array_equal(out[1, :, 32:], x1[1])
+    np.testing.assert_array_equal(out[2, :, :32], neg(x1[2]))
+    np.testing.assert_array_equal(out[2, :, 32:], neg(x2[2]))
+    np.testing.assert_array_equal(out[3, :, :32], x2[3])
+    np.testing.assert_array_equal(out[3, :, 32:], neg(x1[3]))
+
+
+def test_rope_matches_the_fp64_rotation_within_rounding():
+    """Against a rotation in fp64 of the same bf16 inputs by the same
+    (float32) cos/sin: the binary32 steps err by at most 2^-23 of the
+    products' magnitude, the bf16 rounding by half an ulp (at most 2^-8 of
+    the result, at the bottom of a binade)."""
+    rng = np.random.default_rng(62)
+    n, hkv, d = 40, 8, 64
+    rows = _bf16_rows(rng, (n, hkv, d))
+    theta = 10000.0 ** (-np.arange(d // 2) / (d // 2))
+    cs = _rope_table(np.arange(300)[:, None] * theta[None, :])
+    pos = rng.integers(0, 300, n).astype(np.int32)
+    out, bad = oracle.rope(rows, pos, cs)
+    assert bad == 0
+    x = W.bf16_to_f64(rows)
+    c = cs[pos, 0].astype(np.float64)[:, None, :]
+    s = cs[pos, 1].astype(np.float64)[:, None, :]
+    x1, x2 = x[..., :32], x[..., 32:]
+    y = np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+    mag = np.concatenate([np.abs(x1 * c) + np.abs(x2 * s),
+                          np.abs(x2 * c) + np.abs(x1 * s)], axis=-1)
+    got = W.bf16_to_f64(out)
+    assert (np.abs(got - y) <= 2.0 ** -8 * np.abs(y) + 2.0 ** -22 * mag).all()
+    # and not looser than that: some elements need more than a quarter ulp
+    assert (np.abs(got - y) > 2.0 ** -10 * np.abs(y)).any()
+    # a rotation keeps the length of every pair (up to the same rounding)
+    n_in = x1 ** 2 + x2 ** 2
+    n_out = got[..., :32] ** 2 + got[..., 32:] ** 2
+    np.testing.assert_allclose(n_out, n_in, rtol=2.0 ** -6, atol=1e-6)
+
+
+def test_rope_positions_outside_the_table_are_left_alone_and_counted():
+    rng = np.random.default_rng(63)
+    rows = _bf16_rows(rng, (3, 2, 64))
+    cs = _rope_table(rng.random((4, 32)))
+    out, bad = oracle.rope(rows, np.array([-1, 2, 4], np.int32), cs)
+    assert bad == 2
+    np.testing.assert_array_equal(out[0], rows[0])
+    np.testing.assert_array_equal(out[2], rows[2])
+    assert not np.array_equal(out[1], rows[1])
+
+
+def test_kv_append_rope_rotates_k_and_not_v():
+    rng = np.random.default_rng(64)
+    wl = W.decode_workload([5, 40], seed=65)
+    cs = _rope_table(rng.random((64, 32)) * 6.0)
+    pos = (wl.context_lens - 1).astype(np.int32)
+    kp, vp, bad, bad_pos = oracle.kv_append_rope(
+        wl.k_new, wl.v_new, wl.slot_mapping, pos, cs, wl.k_pool, wl.v_pool)
+    assert bad == 0 and bad_pos == 0
+    k_rot, _ = oracle.rope(wl.k_new, pos, cs)
+    kp2, vp2, _ = oracle.kv_append(k_rot, wl.v_new, wl.slot_mapping,
+                                   wl.k_pool, wl.v_pool)
+    np.testing.assert_array_equal(kp, kp2)
+    np.testing.assert_array_equal(vp, vp2)
+    _, vp3, _ = oracle.kv_append(wl.k_new, wl.v_new, wl.slot_mapping,
+                                 wl.k_pool, wl.v_pool)
+    np.testing.assert_array_equal(vp, vp3)
