@@ -54,6 +54,8 @@
  *       TV_DEVERR_POOL_EMPTY   the page pool had too few free pages for a
  *                              sequence (tv_pool_append_slots)
  *       TV_DEVERR_BAD_SEQ      a fork or release named a bad sequence
+ *       TV_DEVERR_BAD_POSITION a RoPE position outside the cos/sin table;
+ *                              that K row is written unrotated
  *   - Outputs must not alias inputs.
  *   - Return: TV_OK, or an error status; TV_ERR_CUDA means the launch failed
  *     (tv_last_cuda_error() gives the CUDA error code).
@@ -84,7 +86,8 @@ enum {
   TV_DEVERR_TIMEOUT = 1u << 3,
   TV_DEVERR_BAD_QUERY = 1u << 4,
   TV_DEVERR_POOL_EMPTY = 1u << 5,
-  TV_DEVERR_BAD_SEQ = 1u << 6
+  TV_DEVERR_BAD_SEQ = 1u << 6,
+  TV_DEVERR_BAD_POSITION = 1u << 7
 };
 
 /* Human-readable name of a status. Never NULL. */
@@ -113,6 +116,34 @@ tv_status tv_kv_append(const void* k_new, const void* v_new,
                        void* k_pool, void* v_pool, int64_t num_pages,
                        int num_kv_heads, int head_dim, int page_size,
                        uint32_t* err, void* stream);
+
+/*
+ * tv_kv_append_rope -- tv_kv_append with every new K row rotated at its
+ * position first ([P1] "Llama 3.2 1B架构拆解": RoPE injects the position into
+ * Q and K by rotation; V is not rotated).  The pages give no pairing, angles
+ * or arithmetic; this library's reading:
+ *   - dimension i is rotated with i + head_dim/2 (rotate-half pairing);
+ *   - rope_cos_sin  [rope_max_position][2][head_dim/2] fp32, device, 16-byte
+ *                   aligned: cos (row 0) and sin (row 1) of each pair's
+ *                   angle at each position (any base or scaling is the
+ *                   caller's);
+ *   - with x1 = k[i], x2 = k[i + head_dim/2], c, s the table entries:
+ *       k'[i]            = bf16_rn(fl(fl(x1 c) - fl(x2 s)))
+ *       k'[i + head_dim/2] = bf16_rn(fl(fl(x2 c) + fl(x1 s)))
+ *     fl = one binary32 rounding (no fused multiply-add), bf16_rn = round
+ *     to nearest even.
+ *   positions   [num_tokens] int32: the token's position in its sequence; a
+ *               position outside [0, rope_max_position) writes the row
+ *               unrotated and flags TV_DEVERR_BAD_POSITION
+ * Other arguments and behaviour as tv_kv_append.
+ */
+tv_status tv_kv_append_rope(const void* k_new, const void* v_new,
+                            const int32_t* slot_mapping,
+                            const int32_t* positions, int64_t num_tokens,
+                            void* k_pool, void* v_pool, int64_t num_pages,
+                            int num_kv_heads, int head_dim, int page_size,
+                            const float* rope_cos_sin, int rope_max_position,
+                            uint32_t* err, void* stream);
 
 /*
  * tv_paged_decode -- one query per sequence at position context_lens[s]-1
@@ -162,6 +193,20 @@ tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
                                  int head_dim, int page_size,
                                  int64_t num_pages, float scale,
                                  uint32_t* err, void* stream);
+
+/*
+ * tv_paged_decode_append_rope -- tv_paged_decode_append with the new K row
+ * of every sequence rotated at its position context_lens[s]-1 (the RoPE of
+ * tv_kv_append_rope, same table and arithmetic) before it enters the pool
+ * and the attention; q is used as given (rotated by the caller).
+ */
+tv_status tv_paged_decode_append_rope(
+    void* out, const void* q, const void* k_new, const void* v_new,
+    void* k_pool, void* v_pool, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+    int64_t num_pages, float scale, const float* rope_cos_sin,
+    int rope_max_position, uint32_t* err, void* stream);
 
 /*
  * tv_decode_workspace_size -- bytes of device workspace that

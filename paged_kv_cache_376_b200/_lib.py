@@ -28,6 +28,7 @@ DEVERR_TIMEOUT = 1 << 3
 DEVERR_BAD_QUERY = 1 << 4
 DEVERR_POOL_EMPTY = 1 << 5
 DEVERR_BAD_SEQ = 1 << 6
+DEVERR_BAD_POSITION = 1 << 7
 
 # (name, restype, argtypes) of every symbol include/tv.h declares
 _P, _I, _I64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
@@ -37,8 +38,13 @@ SIGNATURES = {
     "tv_version": (_I, []),
     "tv_kv_append": (_I, [_P, _P, _P, _I64, _P, _P, _I64, _I, _I, _I, _P,
                           _P]),
+    "tv_kv_append_rope": (_I, [_P, _P, _P, _P, _I64, _P, _P, _I64, _I, _I,
+                               _I, _P, _I, _P, _P]),
     "tv_paged_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                              _I64, _F, _P, _P]),
+    "tv_paged_decode_append_rope": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P,
+                                         _I, _I, _I, _I, _I, _I64, _F, _P, _I,
+                                         _P, _P]),
     "tv_paged_decode_append": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I,
                                     _I, _I, _I, _I, _I64, _F, _P, _P]),
     "tv_paged_decode_split": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I,
@@ -146,6 +152,68 @@ def tv_kv_append(k_new, v_new, slot_mapping, k_pool, v_pool, err=None,
                             k_new.shape[0], _ptr(k_pool), _ptr(v_pool),
                             num_pages, hkv, d, page_size, _ptr(err),
                             _stream(stream)), "tv_kv_append")
+
+
+def _rope_table(cos_sin, d):
+    _cuda(cos_sin, torch.float32, "rope_cos_sin")
+    if cos_sin.dim() != 3 or tuple(cos_sin.shape[1:]) != (2, d // 2):
+        raise ValueError("rope_cos_sin must be [max_position][2][head_dim//2]")
+    return cos_sin.shape[0]
+
+
+def tv_kv_append_rope(k_new, v_new, slot_mapping, positions, k_pool, v_pool,
+                      cos_sin, err=None, stream=None):
+    """tv_kv_append with each K row rotated at positions[t] (RoPE, angles
+    from cos_sin [max_position][2][D/2] fp32: cos row, sin row)."""
+    lib = load()
+    bf = torch.bfloat16
+    _cuda(k_new, bf, "k_new"), _cuda(v_new, bf, "v_new")
+    _cuda(k_pool, bf, "k_pool"), _cuda(v_pool, bf, "v_pool")
+    _cuda(slot_mapping, torch.int32, "slot_mapping")
+    _cuda(positions, torch.int32, "positions")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    if v_pool.shape != k_pool.shape or k_new.shape != v_new.shape:
+        raise ValueError("K/V shape mismatch")
+    if k_new.shape[1:] != (hkv, d) or slot_mapping.shape != k_new.shape[:1] \
+            or positions.shape != slot_mapping.shape:
+        raise ValueError("k_new must be [T][Hkv][D] with slot_mapping and "
+                         "positions [T]")
+    max_pos = _rope_table(cos_sin, d)
+    _check(lib.tv_kv_append_rope(
+        _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(positions),
+        k_new.shape[0], _ptr(k_pool), _ptr(v_pool), num_pages, hkv, d,
+        page_size, _ptr(cos_sin), max_pos, _ptr(err), _stream(stream)),
+        "tv_kv_append_rope")
+
+
+def tv_paged_decode_append_rope(out, q, k_new, v_new, k_pool, v_pool,
+                                block_tables, context_lens, scale, cos_sin,
+                                err=None, stream=None):
+    """tv_paged_decode_append with each sequence's new K row rotated at its
+    position context_len-1 (RoPE, table as tv_kv_append_rope)."""
+    lib = load()
+    bf = torch.bfloat16
+    for n, t in (("out", out), ("q", q), ("k_new", k_new), ("v_new", v_new),
+                 ("k_pool", k_pool), ("v_pool", v_pool)):
+        _cuda(t, bf, n)
+    _cuda(block_tables, torch.int32, "block_tables")
+    _cuda(context_lens, torch.int32, "context_lens")
+    if err is not None:
+        _cuda(err, torch.int32, "err")
+    num_pages, page_size, hkv, d = k_pool.shape
+    b, hq, _ = q.shape
+    if out.shape != q.shape or block_tables.shape[0] != b or \
+            k_new.shape != (b, hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch")
+    max_pos = _rope_table(cos_sin, d)
+    _check(lib.tv_paged_decode_append_rope(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+        _ptr(v_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), b, hq, hkv, d, page_size, num_pages, float(scale),
+        _ptr(cos_sin), max_pos, _ptr(err), _stream(stream)),
+        "tv_paged_decode_append_rope")
 
 
 def tv_paged_decode(out, q, k_pool, v_pool, block_tables, context_lens,

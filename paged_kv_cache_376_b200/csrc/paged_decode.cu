@@ -30,7 +30,8 @@
 //    compute the new token's K,V, append them, then attend): the warp that
 //    owns the page holding position context_len-1 writes the new token's row
 //    of its KV head into the pool and into its staged copy of that page, so
-//    the step is one launch and the new row is never read back from HBM.
+//    the step is one launch and the new row is never read back from HBM;
+//    with a cos/sin table it rotates that K row by RoPE first.
 #include "tv_decode.cuh"
 #include "tv_device.cuh"
 #include "tv_kernels.h"
@@ -120,6 +121,29 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
             (lane < 8 ? a.k_new : a.v_new) +
             ((size_t)seq * gridDim.x + kvh) * kD + chk * 8;
         app_row = *reinterpret_cast<const uint4*>(src);
+      }
+      if (a.rope_cos_sin) {
+        // RoPE of the new K row at its position: lane c < 8 holds dimensions
+        // 8c .. 8c+7, so lanes c and c ^ 4 hold the two halves of the pairs
+        // (i, i + 32); each rotates its pair and keeps its own half
+        uint4 other;
+        other.x = __shfl_xor_sync(0xffffffffu, app_row.x, 4);
+        other.y = __shfl_xor_sync(0xffffffffu, app_row.y, 4);
+        other.z = __shfl_xor_sync(0xffffffffu, app_row.z, 4);
+        other.w = __shfl_xor_sync(0xffffffffu, app_row.w, 4);
+        const int pos = ctx - 1;
+        if (lane < 8) {
+          if (pos < a.rope_max_position) {
+            float c8[8], s8[8];
+            rope_load8(a.rope_cos_sin, pos, 8 * (lane & 3), c8, s8);
+            uint4 lo = lane < 4 ? app_row : other;
+            uint4 hi = lane < 4 ? other : app_row;
+            rope_rotate8(lo, hi, c8, s8);
+            app_row = lane < 4 ? lo : hi;
+          } else if (lane == 0) {
+            flag_error(a.err, DEVERR_BAD_POSITION);
+          }
+        }
       }
     }
   }

@@ -162,6 +162,30 @@ tv_status tv_kv_append(const void* k_new, const void* v_new,
       static_cast<cudaStream_t>(stream)));
 }
 
+tv_status tv_kv_append_rope(const void* k_new, const void* v_new,
+                            const int32_t* slot_mapping,
+                            const int32_t* positions, int64_t num_tokens,
+                            void* k_pool, void* v_pool, int64_t num_pages,
+                            int num_kv_heads, int head_dim, int page_size,
+                            const float* rope_cos_sin, int rope_max_position,
+                            uint32_t* err, void* stream) {
+  if (num_tokens < 0 || num_pages <= 0 || num_kv_heads <= 0)
+    return TV_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || !page_size_ok(page_size))
+    return TV_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return TV_OK;
+  if (!k_new || !v_new || !slot_mapping || !positions || !k_pool ||
+      !v_pool || !rope_cos_sin || rope_max_position <= 0)
+    return TV_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) ||
+      !aligned16(v_pool) || !aligned16(rope_cos_sin))
+    return TV_ERR_INVALID_ARG;
+  return cuda_status(tv::launch_kv_append_rope(
+      k_new, v_new, slot_mapping, positions, num_tokens, k_pool, v_pool,
+      num_pages * page_size, num_kv_heads, rope_cos_sin, rope_max_position,
+      err, static_cast<cudaStream_t>(stream)));
+}
+
 // Device workspace of the work-balanced decode: per-item counters, then two
 // partial-result slots per warp of the persistent grid.
 struct BalancedWorkspace {
@@ -204,7 +228,9 @@ static tv_status decode_common(void* out, float* partial_out,
                                int partition_tokens, int max_partitions,
                                bool split, uint32_t* err, void* stream,
                                const BalancedWorkspace* ws = nullptr,
-                               const int32_t* grown = nullptr) {
+                               const int32_t* grown = nullptr,
+                               const float* rope_cos_sin = nullptr,
+                               int rope_max_position = 0) {
   tv_status st =
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
   if (st != TV_OK) return st;
@@ -259,6 +285,8 @@ static tv_status decode_common(void* out, float* partial_out,
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.grown = grown;
+  a.rope_cos_sin = rope_cos_sin;
+  a.rope_max_position = rope_max_position;
   a.err = err;
   a.max_blocks_per_seq = max_blocks_per_seq;
   a.num_q_heads = num_q_heads;
@@ -325,6 +353,23 @@ tv_status tv_paged_decode_append(void* out, const void* q, const void* k_new,
                        block_tables, max_blocks_per_seq, context_lens,
                        num_seqs, num_q_heads, num_kv_heads, head_dim,
                        page_size, num_pages, scale, 0, 1, false, err, stream);
+}
+
+tv_status tv_paged_decode_append_rope(
+    void* out, const void* q, const void* k_new, const void* v_new,
+    void* k_pool, void* v_pool, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+    int64_t num_pages, float scale, const float* rope_cos_sin,
+    int rope_max_position, uint32_t* err, void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new || !rope_cos_sin ||
+                       !aligned16(rope_cos_sin) || rope_max_position <= 0))
+    return TV_ERR_INVALID_ARG;
+  return decode_common(out, nullptr, nullptr, q, k_new, v_new, k_pool, v_pool,
+                       block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       page_size, num_pages, scale, 0, 1, false, err, stream,
+                       nullptr, nullptr, rope_cos_sin, rope_max_position);
 }
 
 tv_status tv_decode_workspace_size(int num_seqs, int num_q_heads,

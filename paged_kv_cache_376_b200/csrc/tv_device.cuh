@@ -45,6 +45,48 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ---- RoPE of one 8-element chunk pair ---------------------------------------
+// lo holds dimensions d0 .. d0+7 of a head (d0 < 32) and hi the dimensions
+// d0+32 .. d0+39; cos8 / sin8 the table entries of pairs d0 .. d0+7.  Rotates
+// each pair (x1, x2) to (x1 c - x2 s, x2 c + x1 s) with one binary32
+// rounding per product and per sum (no fused multiply-add), then rounds to
+// bf16 (nearest even).
+__device__ __forceinline__ void rope_rotate8(uint4& lo, uint4& hi,
+                                             const float (&cos8)[8],
+                                             const float (&sin8)[8]) {
+  uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
+  uint32_t b[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float y1[2], y2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float x1 = k ? bf16_hi(a[w]) : bf16_lo(a[w]);
+      const float x2 = k ? bf16_hi(b[w]) : bf16_lo(b[w]);
+      const float c = cos8[2 * w + k], s = sin8[2 * w + k];
+      y1[k] = __fsub_rn(__fmul_rn(x1, c), __fmul_rn(x2, s));
+      y2[k] = __fadd_rn(__fmul_rn(x2, c), __fmul_rn(x1, s));
+    }
+    a[w] = pack_bf16x2(y1[0], y1[1]);
+    b[w] = pack_bf16x2(y2[0], y2[1]);
+  }
+  lo = make_uint4(a[0], a[1], a[2], a[3]);
+  hi = make_uint4(b[0], b[1], b[2], b[3]);
+}
+// cos / sin of pairs d0 .. d0+7 at `pos` from a [positions][2][32] table
+// (16-byte aligned, d0 a multiple of 8).
+__device__ __forceinline__ void rope_load8(const float* table, int pos, int d0,
+                                           float (&cos8)[8],
+                                           float (&sin8)[8]) {
+  const float4* c = reinterpret_cast<const float4*>(table + (size_t)pos * 64 + d0);
+  const float4* s = reinterpret_cast<const float4*>(table + (size_t)pos * 64 + 32 + d0);
+  const float4 c0 = __ldg(c), c1 = __ldg(c + 1), s0 = __ldg(s), s1 = __ldg(s + 1);
+  cos8[0] = c0.x; cos8[1] = c0.y; cos8[2] = c0.z; cos8[3] = c0.w;
+  cos8[4] = c1.x; cos8[5] = c1.y; cos8[6] = c1.z; cos8[7] = c1.w;
+  sin8[0] = s0.x; sin8[1] = s0.y; sin8[2] = s0.z; sin8[3] = s0.w;
+  sin8[4] = s1.x; sin8[5] = s1.y; sin8[6] = s1.z; sin8[7] = s1.w;
+}
+
 // ---- fast base-2 exponent / logarithm (hardware approximations) -----------
 // ex2.approx: relative error ~2^-22, ex2(-inf) = +0.  lg2.approx likewise.
 __device__ __forceinline__ float fast_exp2(float x) {

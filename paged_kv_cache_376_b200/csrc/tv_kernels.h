@@ -24,6 +24,9 @@ struct DecodeArgs {
   // reservation grew (tv_decode_step only)
   const int32_t* grown;
   uint32_t* err;                 // nullable
+  // fused append only: RoPE of the new K row at position ctx-1 (nullable)
+  const float* rope_cos_sin;     // [rope_max_position][2][32] fp32
+  int rope_max_position;
   int max_blocks_per_seq;
   int num_q_heads;
   int num_pages;
@@ -56,6 +59,7 @@ cudaError_t launch_paged_decode(const DecodeArgs& a, const CUtensorMap& tk,
 // Device page pool (page_pool.cu).  Error bits beyond those of tv_device.cuh.
 constexpr uint32_t DEVERR_POOL_EMPTY = 1u << 5;  // too few free pages
 constexpr uint32_t DEVERR_BAD_SEQ = 1u << 6;     // bad fork / release index
+constexpr uint32_t DEVERR_BAD_POSITION = 1u << 7;  // RoPE position off the table
 constexpr int kPoolMaxSeqs = 1024;               // one thread per sequence
 
 cudaError_t launch_pool_init(int32_t* state, int num_pages, int page_size,
@@ -81,6 +85,15 @@ cudaError_t launch_pool_release(int32_t* state, int num_pages, int32_t* bt,
 cudaError_t launch_wait_selftest(uint32_t* err, unsigned long long limit_ns,
                                  unsigned long long* waited_ns,
                                  cudaStream_t stream);
+
+cudaError_t launch_kv_append_rope(const void* k_new, const void* v_new,
+                                  const int32_t* slot_mapping,
+                                  const int32_t* positions, int64_t num_tokens,
+                                  void* k_pool, void* v_pool,
+                                  int64_t num_slots, int num_kv_heads,
+                                  const float* rope_cos_sin,
+                                  int rope_max_position, uint32_t* err,
+                                  cudaStream_t stream);
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new,
                              const int32_t* slot_mapping, int64_t num_tokens,

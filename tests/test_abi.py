@@ -108,6 +108,26 @@ def test_prefill_refuses_a_scale_that_is_not_positive(lib):
                                     None) == 1, scale
 
 
+def test_rope_calls_need_a_table(lib):
+    p = _fake()
+    unaligned = _fake(0x10008)
+    # no table, a misaligned table, an empty table
+    for tab, npos in ((None, 8), (unaligned, 8), (p, 0)):
+        assert lib.tv_kv_append_rope(p, p, p, p, 4, p, p, 10, 8, 64, 16, tab,
+                                     npos, None, None) == 1
+        assert lib.tv_paged_decode_append_rope(
+            p, p, p, p, p, p, p, 4, p, 1, 32, 8, 64, 16, 10, 0.125, tab, npos,
+            None, None) == 1
+    # no positions
+    assert lib.tv_kv_append_rope(p, p, p, None, 4, p, p, 10, 8, 64, 16, p, 8,
+                                 None, None) == 1
+    # head_dim 128 is not supported
+    assert lib.tv_kv_append_rope(p, p, p, p, 4, p, p, 10, 8, 128, 16, p, 8,
+                                 None, None) == 2
+    assert lib.tv_kv_append_rope(None, None, None, None, 0, p, p, 10, 8, 64,
+                                 16, None, 0, None, None) == 0
+
+
 def test_pool_state_size_includes_the_growth_marks(lib):
     """TV_POOL_STATE_INTS(np) = 4 + 4 np + TV_POOL_MAX_SEQS (include/tv.h);
     the binding sizes and checks state arrays by the same rule."""
