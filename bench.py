@@ -609,7 +609,10 @@ def run_tv(args, rank, world, local_rank):
             "bound": bound, "achieved": round(kern_per_launch, 2),
             "peak": peak, "unit": unit, "frac": round(kern_per_launch / peak,
                                                       4),
-            "peak_source": f"{peak_src} ({key})",
+            "peak_source": (f"{peak_src} ({key})" if peak_src == "measured"
+                            or bound == "hbm" else
+                            f"{peak_src} (bf16 burst figure; the fallback "
+                            "has no sustained one)"),
             "kernel": kernel_name,
             "kernel_ms": round(kern_ms_max, 6),
             "traffic": _traffic(kernel_name, wl.name),
