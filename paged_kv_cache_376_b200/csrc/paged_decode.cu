@@ -18,11 +18,14 @@
 //    one mbarrier per slot; warp w takes pages w, w+4, w+8, ... so no warp
 //    ever waits for another until the final combine.  Block-table entries
 //    are prefetched 32 at a time, one per lane, ahead of the TMA issue.
-//  * Inside a warp: lane = 8*g + c; lane-group g owns tokens g, g+4, g+8,
-//    g+12 of the page, lane c owns head dims [8c, 8c+8).  QK partial dots
-//    are summed across the 8 lanes of a group with xor-shuffles; the softmax
-//    is online per page in base 2 (q is pre-scaled by scale*log2(e)): one
-//    max and one rescale per page, not per token.
+//  * Per page the G query heads need S^T = K Q^T and O^T += V^T P^T: dense
+//    products over 64 dims and 16 tokens, which each warp runs on the tensor
+//    cores as m16n8k16 bf16 products with fp32 accumulation (4 for the
+//    scores, 8 for P.V with P split into two bf16 terms), the page slices
+//    read by ldmatrix from the 128-byte-swizzled TMA boxes.  Unpacking bf16
+//    to fp32 and reducing dot products across lanes, which made up most of
+//    the instructions of an fp32 FMA formulation, disappear.  The softmax is
+//    online per page in base 2: one max and (lazily) one rescale per page.
 //  * The split variant writes the normalised partial output and the natural
 //    log-sum-exp of each 512-token (or any multiple of 16) partition; the
 //    merge kernel (split_merge.cu) combines them.
@@ -50,7 +53,7 @@ constexpr float kLazy = 8.f;   // log2 of the growth the running sums allow
 
 template <int kStages>
 struct DecodeSmem {
-  alignas(128) uint8_t ring[kWarps][kStages][kStageBytes];
+  alignas(1024) uint8_t ring[kWarps][kStages][kStageBytes];
   alignas(8) uint64_t full[kWarps][kStages];
 };
 
@@ -78,8 +81,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int part = kSplit ? blockIdx.z : 0;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int grp = lane >> 3;   // token sub-group
-  const int chk = lane & 7;    // 16-byte chunk of the head dim
+  const int chk = lane & 7;    // 16-byte chunk of the appended row
 
   // ---- token range of this CTA --------------------------------------------
   // a decode step (tv_decode_step) treats a sequence whose context did not
@@ -155,36 +157,63 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   }
   __syncwarp();
 
-  // ---- q for the G heads of this KV head, pre-scaled by scale*log2(e) -----
-  // Element pairs (2i, 2i+1) of this lane's 8-element chunk, as float2 so
-  // the dot products run on the packed fp32x2 FMA pipe.  Position h holds
-  // head h ^ rs_mask (the order reduce_scatter8 expects).
-  const int qmask = rs_mask<G>(chk);
-  float2 q2[G][4];
+  // ---- warp-level tensor-core layout ---------------------------------------
+  // Per page and KV head the work is two small dense products for the G
+  // query heads of the group: S^T = K Q^T (16 tokens x G heads, contraction
+  // over the 64 dims) and O^T += V^T P^T (64 dims x G heads, contraction over
+  // the 16 tokens), each as m16n8k16 bf16 products with fp32 accumulation,
+  // heads padded to the 8 columns of the product.  Lane = 4 * g + c:
+  //  * S^T fragment: tokens g and g + 8, heads 2c and 2c + 1;
+  //  * O^T fragment of dim tile t: dims 16t + g and 16t + g + 8, the same
+  //    heads 2c, 2c + 1, so the running max / sum of a lane's heads (and
+  //    their rescaling of O) never leave the lane.
+  const int g = lane >> 2;
+  const int c = lane & 3;
+  const bool hv0 = 2 * c < G, hv1 = 2 * c + 1 < G;   // real heads of the lane
+
+  // q of head g as the B operand of S^T = K Q^T: dims 16k + 2c, +1 (b0) and
+  // 16k + 2c + 8, +9 (b1), unscaled bf16; padded heads are zero.
+  uint32_t qb[4][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + ((size_t)seq * a.num_q_heads + kvh * G + (g < G ? g : 0)) * kD);
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint4 v = *reinterpret_cast<const uint4*>(
-        a.q + ((size_t)seq * a.num_q_heads + kvh * G + (h ^ qmask)) * kD +
-        chk * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      q2[h][i] = make_float2(bf16_lo(w[i]) * a.scale_log2,
-                             bf16_hi(w[i]) * a.scale_log2);
+    for (int k = 0; k < 4; ++k) {
+      qb[k][0] = g < G ? __ldg(qrow + 8 * k + c) : 0u;
+      qb[k][1] = g < G ? __ldg(qrow + 8 * k + c + 4) : 0u;
+    }
   }
-
-  // After the reduce-scatter below, lane chunk c holds the score of head
-  // c >> kShift (lanes that share a head hold the same value); head h is
-  // read from lane (group, h << kShift).
-  constexpr int kShift = G == 8 ? 0 : G == 4 ? 1 : G == 2 ? 2 : 3;
-  const int my_head = chk >> kShift;
-
-  float m_run = -INFINITY, l_run = 0.f;   // for head my_head
-  float2 acc2[G][4];                      // all heads, this lane's 8 dims
+  // ldmatrix row addresses inside a 2 KB page slice stored with the 128-byte
+  // swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)).  K: matrices
+  // (rows 0-7 | 8-15) x (chunk 2k | 2k+1) in A-fragment order; V, loaded
+  // transposed: (chunk 2t | 2t+1) x (rows 0-7 | 8-15).
+  uint32_t koff[4], voff[4];
+  {
+    const int mi = lane >> 3, r7 = lane & 7;
+    const int kr = r7 + 8 * (mi & 1), vr = r7 + 8 * (mi >> 1);
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+    for (int k = 0; k < 4; ++k) {
+      koff[k] = kr * kRowBytes + (((2 * k + (mi >> 1)) ^ r7) << 4);
+      voff[k] = vr * kRowBytes + (((2 * k + (mi & 1)) ^ r7) << 4);
+    }
+  }
+  // P^T as the B operand of the P.V product: lane (g, c) needs P of tokens
+  // 2c, 2c+1 (and + 8) for head g, held by lanes 8c + g/2 and 8c + 4 + g/2
+  // as the (head 2c', 2c'+1) halves of a bf16 pair; the byte permutation
+  // picks half g & 1 of each.
+  const int src_a = 8 * c + (g >> 1), src_b = src_a + 4;
+  const uint32_t half_sel = (g & 1) ? 0x7632u : 0x5410u;
+
+  // running max (base 2, scaled) / sum per head of the lane; padded heads
+  // start at +inf so their probabilities are exp2(-inf) = 0
+  float m0 = hv0 ? -INFINITY : INFINITY, m1 = hv1 ? -INFINITY : INFINITY;
+  float l0 = 0.f, l1 = 0.f;
+  float acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc2[h][i] = make_float2(0.f, 0.f);
+  for (int t = 0; t < 4; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+  const float sl = a.scale_log2;
 
   // Pool blocks of this warp's 16-token blocks, 32 per batch, one per lane
   // (-1 when the block-table entry is not a page of the pool).
@@ -246,96 +275,108 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     if (kAppend && i == app_i) {
       // the staged page now gets the new row; the pool keeps it for later
       if (page_ok && lane < 16) {
-        uint8_t* dst = &sm.ring[warp][stage][(lane < 8 ? 0 : kSliceBytes) +
-                                             app_r * kRowBytes + chk * 16];
+        const int ch = lane & 7;
+        uint8_t* dst = (lane < 8 ? kbase : vbase) + app_r * kRowBytes +
+                       ((ch ^ (app_r & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = app_row;
         __nv_bfloat16* pool = lane < 8 ? a.k_pool_w : a.v_pool_w;
         *reinterpret_cast<uint4*>(
             pool + (((size_t)pid * kPS + app_r) * gridDim.x + kvh) * kD +
-            chk * 8) = app_row;
+            ch * 8) = app_row;
       }
       __syncwarp();
     }
     if (!full_page) {
       // Rows past the range (or the whole of a bad page) get p = 0; zero
-      // their V so that 0 * a stale NaN never reaches the sum.  Each lane
-      // clears exactly the rows and chunk it reads below.
+      // their V so that 0 * a stale NaN never reaches the sum.
 #pragma unroll
-      for (int r = grp; r < kPS; r += 4)
+      for (int e = lane; e < kPS * 8; e += 32) {
+        const int r = e >> 3;
         if (!(page_ok && page_tok0 + r < tok_end))
-          *reinterpret_cast<uint4*>(vbase + r * kRowBytes + chk * 16) =
+          *reinterpret_cast<uint4*>(vbase + r * kRowBytes + (e & 7) * 16) =
               make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+    const uint32_t kb = smem_u32(kbase), vb = smem_u32(vbase);
+
+    // ---- scores S^T = K Q^T: tokens g, g+8 x heads 2c, 2c+1 ----------------
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t ka[4];
+      ldsm_x4(kb + koff[k], ka);
+      mma_bf16_16816(s, ka, qb[k][0], qb[k][1]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] *= sl;
+    if (!full_page) {
+      const bool t0 = page_ok && page_tok0 + g < tok_end;
+      const bool t1 = page_ok && page_tok0 + g + 8 < tok_end;
+      s[0] = t0 ? s[0] : -INFINITY;
+      s[1] = t0 ? s[1] : -INFINITY;
+      s[2] = t1 ? s[2] : -INFINITY;
+      s[3] = t1 ? s[3] : -INFINITY;
     }
 
-    // ---- scores: token it*4+grp, head my_head ---------------------------------
-    float s[4];
+    // ---- online softmax, once per page, with a lazy offset -----------------
+    // The offset only moves when a page maximum exceeds it by more than
+    // 2^kLazy (base 2): exp2(s - m) then stays below 2^kLazy, and any offset
+    // gives the same acc / l.
+    float pm0 = fmaxf(s[0], s[2]), pm1 = fmaxf(s[1], s[3]);
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 4 + grp;
-      const uint4 kv =
-          *reinterpret_cast<const uint4*>(kbase + r * kRowBytes + chk * 16);
-      const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-      float2 k2[4];
+    for (int off = 4; off < 32; off <<= 1) {
+      pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, off));
+      pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, off));
+    }
+    if (__any_sync(0xffffffffu, pm0 > m0 + kLazy || pm1 > m1 + kLazy)) {
+      const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
+      // equal offsets (both -inf, or a padded head's +inf) keep the sums
+      const float a0 = n0 == m0 ? 1.f : fast_exp2(m0 - n0);
+      const float a1 = n1 == m1 ? 1.f : fast_exp2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      l0 *= a0;
+      l1 *= a1;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) k2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
-      float part[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float2 d2 = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-        for (int t = 1; t < 4; ++t) d2 = __ffma2_rn(q2[h][t], k2[t], d2);
-        part[h] = d2.x + d2.y;
-      }
-      // reduce-scatter over the 8 lanes of the group (no selects: the q
-      // positions are permuted per lane)
-      s[it] = reduce_scatter8<G>(part);
-      if (!full_page) {
-        const bool valid = page_ok && (page_tok0 + r) < tok_end;
-        s[it] = valid ? s[it] : -INFINITY;
+      for (int t = 0; t < 4; ++t) {
+        acc[t][0] *= a0;
+        acc[t][1] *= a1;
+        acc[t][2] *= a0;
+        acc[t][3] *= a1;
       }
     }
+    const float mu0 = m0 == -INFINITY ? 0.f : m0;
+    const float mu1 = m1 == -INFINITY ? 0.f : m1;
+    const float p0 = fast_exp2(s[0] - mu0), p1 = fast_exp2(s[1] - mu1);
+    const float p2 = fast_exp2(s[2] - mu0), p3 = fast_exp2(s[3] - mu1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
 
-    // ---- online softmax, once per page, with a lazy offset -----------------------
-    // The offset m_run only moves when a page maximum exceeds it by more
-    // than 2^kLazy (base 2): exp2(s - m_run) then stays below 2^kLazy, and
-    // any offset gives the same acc / l.
-    float pm = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
-    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
-    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
-    if (__any_sync(0xffffffffu, pm > m_run + kLazy)) {
-      const float m_new = fmaxf(m_run, pm);
-      const float alpha = fast_exp2(m_run - (m_new == -INFINITY ? 0.f : m_new));
-      m_run = m_new;
-      l_run *= alpha;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float ah = __shfl_sync(0xffffffffu, alpha, h << kShift);
-        const float2 a2 = make_float2(ah, ah);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc2[h][t] = __fmul2_rn(acc2[h][t], a2);
-      }
-    }
-    const float m_use = m_run == -INFINITY ? 0.f : m_run;
+    // ---- P as two bf16 terms (hi + lo, ~16 significant bits) in B layout ---
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    const uint32_t r01 = pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
+    const uint32_t r23 = pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
+    const uint32_t bh0 = __byte_perm(__shfl_sync(0xffffffffu, h01, src_a),
+                                     __shfl_sync(0xffffffffu, h01, src_b),
+                                     half_sel);
+    const uint32_t bh1 = __byte_perm(__shfl_sync(0xffffffffu, h23, src_a),
+                                     __shfl_sync(0xffffffffu, h23, src_b),
+                                     half_sel);
+    const uint32_t bl0 = __byte_perm(__shfl_sync(0xffffffffu, r01, src_a),
+                                     __shfl_sync(0xffffffffu, r01, src_b),
+                                     half_sel);
+    const uint32_t bl1 = __byte_perm(__shfl_sync(0xffffffffu, r23, src_a),
+                                     __shfl_sync(0xffffffffu, r23, src_b),
+                                     half_sel);
 
-    // ---- P.V -------------------------------------------------------------------
+    // ---- O^T += V^T P^T ------------------------------------------------------
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 4 + grp;
-      const float p = fast_exp2(s[it] - m_use);
-      l_run += p;
-      const uint4 vv =
-          *reinterpret_cast<const uint4*>(vbase + r * kRowBytes + chk * 16);
-      const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-      float2 v2[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) v2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float ph = __shfl_sync(0xffffffffu, p, grp * 8 + (h << kShift));
-        const float2 p2 = make_float2(ph, ph);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc2[h][t] = __ffma2_rn(p2, v2[t], acc2[h][t]);
-      }
+    for (int t = 0; t < 4; ++t) {
+      uint32_t va[4];
+      ldsm_x4_trans(vb + voff[t], va);
+      mma_bf16_16816(acc[t], va, bh0, bh1);
+      mma_bf16_16816(acc[t], va, bl0, bl1);
     }
 
     // ---- hand the slot back to the TMA unit ------------------------------------
@@ -356,40 +397,43 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     if (lane == 0) flag_error(a.err, DEVERR_TIMEOUT);
     for (int k = i; k < issued; ++k)
       mbar_wait(smem_u32(&sm.full[warp][k % kStages]), (k / kStages) & 1);
-    m_run = -INFINITY;
-    l_run = 0.f;
+    m0 = hv0 ? -INFINITY : INFINITY;
+    m1 = hv1 ? -INFINITY : INFINITY;
+    l0 = l1 = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int t = 0; t < 4; ++t)
 #pragma unroll
-      for (int t = 0; t < 4; ++t) acc2[h][t] = make_float2(0.f, 0.f);
+      for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
   }
 
-  // ---- reduce over the 4 lane groups ------------------------------------------
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+  // ---- sums over the 8 token lanes (g) of each head -----------------------
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 8);
-      acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 8);
-      acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 16);
-      acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 16);
-    }
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
   __syncthreads();  // every warp is done with its ring
   auto& cb = *reinterpret_cast<Combine<G>*>(smem_raw);
-  if (grp == 0) {
+  if (hv0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int t = 0; t < 4; ++t) {
+      cb.acc[warp][2 * c][16 * t + g] = acc[t][0];
+      cb.acc[warp][2 * c][16 * t + g + 8] = acc[t][2];
+    }
+    if (g == 0) {
+      cb.m[warp][2 * c] = m0;
+      cb.l[warp][2 * c] = l0;
+    }
+  }
+  if (hv1) {
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        cb.acc[warp][h][chk * 8 + 2 * t] = acc2[h][t].x;
-        cb.acc[warp][h][chk * 8 + 2 * t + 1] = acc2[h][t].y;
-      }
-    if ((chk & ((1 << kShift) - 1)) == 0) {
-      cb.m[warp][my_head] = m_run;
-      cb.l[warp][my_head] = l_run;
+    for (int t = 0; t < 4; ++t) {
+      cb.acc[warp][2 * c + 1][16 * t + g] = acc[t][1];
+      cb.acc[warp][2 * c + 1][16 * t + g + 8] = acc[t][3];
+    }
+    if (g == 0) {
+      cb.m[warp][2 * c + 1] = m1;
+      cb.l[warp][2 * c + 1] = l1;
     }
   }
   __syncthreads();
