@@ -33,9 +33,10 @@
 //  * Each warp runs the same page pipeline as paged_decode.cu (a private
 //    ring of kStages TMA-filled page slots, one mbarrier each) straight
 //    across item boundaries, so short items cost no pipeline drain.  At the
-//    first page of an item it takes the item's q (prefetched one item ahead
-//    into shared memory); at the item's last page in its range it finishes
-//    the item.
+//    first page of an item it takes the item's q (fetched one item ahead
+//    into registers); at the item's last page in its range it finishes the
+//    item.  The per-page arithmetic is that of paged_decode.cu: the scores
+//    and P.V of the G heads as warp-level bf16 tensor-core products.
 //  * An item that lies inside one warp's range is written directly.  An
 //    item cut by range boundaries is a set of segments, one per group; each
 //    writes (m, l, acc) for its G heads to its workspace slot (slot 0 for
@@ -70,27 +71,15 @@ constexpr int kSideBytes = 2 * kRowBytes;        // new K row + new V row
 constexpr float kLazy = 8.f;                     // log2 of the allowed growth
 constexpr uint32_t kNoPage = (1u << 26) - 1;     // page word: nothing to load
 
-template <int G>
 struct BalancedSmem {
-  alignas(128) uint8_t ring[kWarps][kStages][kStageBytes];
+  // 1024-byte aligned: the slices are 128-byte-swizzled TMA boxes
+  alignas(1024) uint8_t ring[kWarps][kStages][kStageBytes];
   alignas(128) uint8_t side[kWarps][kStages][kSideBytes];
-  alignas(128) uint8_t q_next[kWarps][G * kRowBytes];  // q of the next item
   alignas(8) uint64_t full[kWarps][kStages];
   int32_t warp_total[kWarps];
   int32_t pre[kMaxBalancedSeqs + 1];
   uint8_t last_valid[kMaxBalancedSeqs];  // tokens in each sequence's last page
 };
-
-// 16-byte global -> shared copy that completes asynchronously (waited for
-// with cp_async_wait_all by the same thread).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src))
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src,
                                           uint32_t bytes, uint32_t bar) {
@@ -110,9 +99,10 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     balanced_decode_kernel(const DecodeArgs a,
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v) {
-  extern __shared__ __align__(128) uint8_t smem_dyn[];
-  uint8_t* smem_raw = smem_dyn + ((128 - (smem_u32(smem_dyn) & 127)) & 127);
-  auto& sm = *reinterpret_cast<BalancedSmem<G>*>(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_dyn[];
+  // 1 KB of slack is requested at launch; align the carve-out by hand.
+  uint8_t* smem_raw = smem_dyn + ((1024 - (smem_u32(smem_dyn) & 1023)) & 1023);
+  auto& sm = *reinterpret_cast<BalancedSmem*>(smem_raw);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -266,26 +256,47 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     if (j < n && lane == 0) issue(q_w[j], seq_issue, j);
   }
 
-  constexpr int kShift = G == 8 ? 0 : G == 4 ? 1 : G == 2 ? 2 : 3;
-  const int qmask = rs_mask<G>(chk);
-
-  // q of sequence s for this warp's KV head (G heads x 128 B, contiguous)
-  // into the warp's q slot, 16 bytes per lane, asynchronously
-  const uint32_t q_slot = smem_u32(&sm.q_next[warp][0]);
-  auto load_q = [&](int seq) {
-    if (seq < B) {
-      const __nv_bfloat16* src =
-          a.q + ((size_t)seq * a.num_q_heads + head * G) * kD;
+  // Warp-level tensor-core layout, as in paged_decode.cu: per page,
+  // S^T = K Q^T and O^T += V^T P^T as m16n8k16 bf16 products (fp32
+  // accumulation, heads padded to 8 columns).  Lane = 4 g + c holds tokens
+  // g, g+8 of the scores and dims 16t + g, +8 of the accumulator, both for
+  // heads 2c and 2c+1.
+  const int g = lane >> 2;
+  const int c = lane & 3;
+  const bool hv0 = 2 * c < G, hv1 = 2 * c + 1 < G;
+  uint32_t koff[4], voff[4];
+  {
+    const int mi = lane >> 3, r7 = lane & 7;
+    const int kr = r7 + 8 * (mi & 1), vr = r7 + 8 * (mi >> 1);
 #pragma unroll
-      for (int k = lane; k < G * 8; k += 32)
-        cp_async16(q_slot + k * 16, src + k * 8);
+    for (int k = 0; k < 4; ++k) {
+      koff[k] = kr * kRowBytes + (((2 * k + (mi >> 1)) ^ r7) << 4);
+      voff[k] = vr * kRowBytes + (((2 * k + (mi & 1)) ^ r7) << 4);
+    }
+  }
+  const int src_a = 8 * c + (g >> 1), src_b = src_a + 4;
+  const uint32_t half_sel = (g & 1) ? 0x7632u : 0x5410u;
+  const float sl = a.scale_log2;
+
+  // q fragments (B operand of the scores, head g of the group) of the next
+  // item, fetched into registers one item ahead
+  uint32_t qn[4][2];
+  auto load_q = [&](int sq) {
+    const bool ok = sq < B && g < G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + ((size_t)(ok ? sq : 0) * a.num_q_heads + head * G +
+               (g < G ? g : 0)) * kD);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      qn[k][0] = ok ? __ldg(qrow + 8 * k + c) : 0u;
+      qn[k][1] = ok ? __ldg(qrow + 8 * k + c + 4) : 0u;
     }
   };
   load_q(seq0);
 
-  float2 q2[G][4];
-  float2 acc2[G][4];
-  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t qb[4][2];
+  float acc[4][4];
+  float m0 = INFINITY, m1 = INFINITY, l0 = 0.f, l1 = 0.f;
   bool seg_at_range_start = true;   // the segment began at x0
   bool seg_at_item_start = true;    // the segment began at page 0
 
@@ -307,27 +318,23 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     // ---- a new item starts: take its q, reset the running state ------------
     if (i == 0 || first_of_item) {
       if (i > 0) ++seq;
-      cp_async_wait_all();
-      __syncwarp();
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint4 qv = *reinterpret_cast<const uint4*>(
-            &sm.q_next[warp][(h ^ qmask) * kRowBytes + chk * 16]);
-        const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          q2[h][t] = make_float2(bf16_lo(w[t]) * a.scale_log2,
-                                 bf16_hi(w[t]) * a.scale_log2);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc2[h][t] = make_float2(0.f, 0.f);
+      for (int k = 0; k < 4; ++k) {
+        qb[k][0] = qn[k][0];
+        qb[k][1] = qn[k][1];
       }
-      m_run = -INFINITY;
-      l_run = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+      // padded heads keep +inf: their probabilities are exp2(-inf) = 0
+      m0 = hv0 ? -INFINITY : INFINITY;
+      m1 = hv1 ? -INFINITY : INFINITY;
+      l0 = l1 = 0.f;
       seg_at_range_start = i == 0;
       seg_at_item_start = first_of_item;
       // this warp's next item is the next sequence, same KV head (fetched
       // even when the range ends first: one spare read of G x 128 bytes)
-      __syncwarp();
       load_q(seq + 1);
     }
 
@@ -345,7 +352,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
         const uint4 row = *reinterpret_cast<const uint4*>(
             &sm.side[warp][stage][(lane < 8 ? 0 : kRowBytes) + chk * 16]);
         *reinterpret_cast<uint4*>(kbase + (lane < 8 ? 0 : kSliceBytes) +
-                                  r * kRowBytes + chk * 16) = row;
+                                  r * kRowBytes + ((chk ^ (r & 7)) << 4)) =
+            row;
         __nv_bfloat16* pool = lane < 8 ? a.k_pool_w : a.v_pool_w;
         *reinterpret_cast<uint4*>(
             pool + (((size_t)pid * kPS + r) * Hkv + head) * kD + chk * 8) =
@@ -356,77 +364,88 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
     if (!full_page) {
       // Rows past the context (or the whole of an unloaded page) get p = 0;
-      // zero their V so that 0 * a stale NaN never reaches the sum.  Each
-      // lane clears exactly the rows and chunk it reads below.
+      // zero their V so that 0 * a stale NaN never reaches the sum.
 #pragma unroll
-      for (int r = grp; r < kPS; r += 4)
+      for (int e = lane; e < kPS * 8; e += 32) {
+        const int r = e >> 3;
         if (!(page_ok && r < valid))
-          *reinterpret_cast<uint4*>(vbase + r * kRowBytes + chk * 16) =
+          *reinterpret_cast<uint4*>(vbase + r * kRowBytes + (e & 7) * 16) =
               make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+    const uint32_t kb = smem_u32(kbase), vb = smem_u32(vbase);
+
+    // ---- scores S^T = K Q^T: tokens g, g+8 x heads 2c, 2c+1 ----------------
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t ka[4];
+      ldsm_x4(kb + koff[k], ka);
+      mma_bf16_16816(s, ka, qb[k][0], qb[k][1]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] *= sl;
+    if (!full_page) {
+      const bool t0 = page_ok && g < valid, t1 = page_ok && g + 8 < valid;
+      s[0] = t0 ? s[0] : -INFINITY;
+      s[1] = t0 ? s[1] : -INFINITY;
+      s[2] = t1 ? s[2] : -INFINITY;
+      s[3] = t1 ? s[3] : -INFINITY;
     }
 
-    // ---- scores: token it*4+grp, head my_head --------------------------------
-    float s[4];
+    // ---- online softmax with a lazy offset ----------------------------------
+    float pm0 = fmaxf(s[0], s[2]), pm1 = fmaxf(s[1], s[3]);
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 4 + grp;
-      const uint4 kv =
-          *reinterpret_cast<const uint4*>(kbase + r * kRowBytes + chk * 16);
-      const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-      float2 k2[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) k2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
-      float part[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float2 d2 = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-        for (int t = 1; t < 4; ++t) d2 = __ffma2_rn(q2[h][t], k2[t], d2);
-        part[h] = d2.x + d2.y;
-      }
-      s[it] = reduce_scatter8<G>(part);
-      if (!full_page) s[it] = (page_ok && r < valid) ? s[it] : -INFINITY;
+    for (int off = 4; off < 32; off <<= 1) {
+      pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, off));
+      pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, off));
     }
-
-    // ---- online softmax with a lazy offset --------------------------------------
-    float pm = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
-    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
-    pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 16));
-    if (__any_sync(0xffffffffu, pm > m_run + kLazy)) {
-      const float m_new = fmaxf(m_run, pm);
-      const float alpha =
-          fast_exp2(m_run - (m_new == -INFINITY ? 0.f : m_new));
-      m_run = m_new;
-      l_run *= alpha;
+    if (__any_sync(0xffffffffu, pm0 > m0 + kLazy || pm1 > m1 + kLazy)) {
+      const float n0 = fmaxf(m0, pm0), n1 = fmaxf(m1, pm1);
+      const float a0 = n0 == m0 ? 1.f : fast_exp2(m0 - n0);
+      const float a1 = n1 == m1 ? 1.f : fast_exp2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      l0 *= a0;
+      l1 *= a1;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float ah = __shfl_sync(0xffffffffu, alpha, h << kShift);
-        const float2 a2 = make_float2(ah, ah);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc2[h][t] = __fmul2_rn(acc2[h][t], a2);
+      for (int t = 0; t < 4; ++t) {
+        acc[t][0] *= a0;
+        acc[t][1] *= a1;
+        acc[t][2] *= a0;
+        acc[t][3] *= a1;
       }
     }
-    const float m_use = m_run == -INFINITY ? 0.f : m_run;
+    const float mu0 = m0 == -INFINITY ? 0.f : m0;
+    const float mu1 = m1 == -INFINITY ? 0.f : m1;
+    const float p0 = fast_exp2(s[0] - mu0), p1 = fast_exp2(s[1] - mu1);
+    const float p2 = fast_exp2(s[2] - mu0), p3 = fast_exp2(s[3] - mu1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
 
-    // ---- P.V ------------------------------------------------------------------
+    // ---- P (bf16 hi + lo) in B layout; O^T += V^T P^T -------------------------
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    const uint32_t r01 = pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
+    const uint32_t r23 = pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
+    const uint32_t bh0 = __byte_perm(__shfl_sync(0xffffffffu, h01, src_a),
+                                     __shfl_sync(0xffffffffu, h01, src_b),
+                                     half_sel);
+    const uint32_t bh1 = __byte_perm(__shfl_sync(0xffffffffu, h23, src_a),
+                                     __shfl_sync(0xffffffffu, h23, src_b),
+                                     half_sel);
+    const uint32_t bl0 = __byte_perm(__shfl_sync(0xffffffffu, r01, src_a),
+                                     __shfl_sync(0xffffffffu, r01, src_b),
+                                     half_sel);
+    const uint32_t bl1 = __byte_perm(__shfl_sync(0xffffffffu, r23, src_a),
+                                     __shfl_sync(0xffffffffu, r23, src_b),
+                                     half_sel);
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 4 + grp;
-      const float pr = fast_exp2(s[it] - m_use);
-      l_run += pr;
-      const uint4 vv =
-          *reinterpret_cast<const uint4*>(vbase + r * kRowBytes + chk * 16);
-      const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-      float2 v2[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) v2[t] = make_float2(bf16_lo(w[t]), bf16_hi(w[t]));
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float ph = __shfl_sync(0xffffffffu, pr, grp * 8 + (h << kShift));
-        const float2 p2 = make_float2(ph, ph);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc2[h][t] = __ffma2_rn(p2, v2[t], acc2[h][t]);
-      }
+    for (int t = 0; t < 4; ++t) {
+      uint32_t va[4];
+      ldsm_x4_trans(vb + voff[t], va);
+      mma_bf16_16816(acc[t], va, bh0, bh1);
+      mma_bf16_16816(acc[t], va, bl0, bl1);
     }
 
     // ---- hand the slot back, issue the page kStages ahead ------------------------
@@ -452,34 +471,32 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
     // ---- the item ends in this range: finish it ---------------------------------
     if (last_of_item || i == n - 1) {
-      float l = l_run;
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      float L0 = l0, L1 = l1;   // sums over the 8 token lanes of each head
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 8);
-          acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 8);
-          acc2[h][t].x += __shfl_xor_sync(0xffffffffu, acc2[h][t].x, 16);
-          acc2[h][t].y += __shfl_xor_sync(0xffffffffu, acc2[h][t].y, 16);
-        }
+      for (int off = 4; off < 32; off <<= 1) {
+        L0 += __shfl_xor_sync(0xffffffffu, L0, off);
+        L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+      }
       const int u = seq * Hkv + head;
       __nv_bfloat16* out_item =
           a.out + ((size_t)seq * a.num_q_heads + head * G) * kD;
       if (seg_at_item_start && last_of_item) {
         // the whole item is in this range
+        const float inv0 = L0 > 0.f ? 1.f / L0 : 0.f;
+        const float inv1 = L1 > 0.f ? 1.f / L1 : 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float lh = __shfl_sync(0xffffffffu, l, h << kShift);
-          if ((h & 3) == grp) {
-            const float inv = lh > 0.f ? 1.f / lh : 0.f;
-            uint4 o;
-            o.x = pack_bf16x2(acc2[h][0].x * inv, acc2[h][0].y * inv);
-            o.y = pack_bf16x2(acc2[h][1].x * inv, acc2[h][1].y * inv);
-            o.z = pack_bf16x2(acc2[h][2].x * inv, acc2[h][2].y * inv);
-            o.w = pack_bf16x2(acc2[h][3].x * inv, acc2[h][3].y * inv);
-            *reinterpret_cast<uint4*>(out_item + h * kD + chk * 8) = o;
+        for (int t = 0; t < 4; ++t) {
+          if (hv0) {
+            out_item[2 * c * kD + 16 * t + g] =
+                __float2bfloat16_rn(acc[t][0] * inv0);
+            out_item[2 * c * kD + 16 * t + g + 8] =
+                __float2bfloat16_rn(acc[t][2] * inv0);
+          }
+          if (hv1) {
+            out_item[(2 * c + 1) * kD + 16 * t + g] =
+                __float2bfloat16_rn(acc[t][1] * inv1);
+            out_item[(2 * c + 1) * kD + 16 * t + g + 8] =
+                __float2bfloat16_rn(acc[t][3] * inv1);
           }
         }
       } else {
@@ -487,20 +504,26 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
         float* slot = a.ws_partials +
                       ((size_t)gw * 2 + (seg_at_range_start ? 0 : 1)) *
                           kSlotFloats;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float mh = __shfl_sync(0xffffffffu, m_run, h << kShift);
-          const float lh = __shfl_sync(0xffffffffu, l, h << kShift);
-          if (lane == 0) {
-            slot[h] = mh;
-            slot[8 + h] = lh;
+        if (hv0) {
+          if (g == 0) {
+            slot[2 * c] = m0;
+            slot[8 + 2 * c] = L0;
           }
-          if ((h & 3) == grp) {
-            float4* dst = reinterpret_cast<float4*>(slot + 16 + h * kD + chk * 8);
-            dst[0] = make_float4(acc2[h][0].x, acc2[h][0].y, acc2[h][1].x,
-                                 acc2[h][1].y);
-            dst[1] = make_float4(acc2[h][2].x, acc2[h][2].y, acc2[h][3].x,
-                                 acc2[h][3].y);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            slot[16 + 2 * c * kD + 16 * t + g] = acc[t][0];
+            slot[16 + 2 * c * kD + 16 * t + g + 8] = acc[t][2];
+          }
+        }
+        if (hv1) {
+          if (g == 0) {
+            slot[2 * c + 1] = m1;
+            slot[8 + 2 * c + 1] = L1;
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            slot[16 + (2 * c + 1) * kD + 16 * t + g] = acc[t][1];
+            slot[16 + (2 * c + 1) * kD + 16 * t + g + 8] = acc[t][3];
           }
         }
         __threadfence();
@@ -647,13 +670,13 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
 
 // Four CTAs of G <= 4 must fit in one SM's 228 KB (1 KB of it reserved per
 // CTA) so that 16 warps stream per SM.
-static_assert(4 * (sizeof(BalancedSmem<4>) + 128 + 1024) <= 228 * 1024,
+static_assert(4 * (sizeof(BalancedSmem) + 1024 + 1024) <= 228 * 1024,
               "shared memory of the balanced decode exceeds 4 CTAs per SM");
 
 template <int G, bool kAppend>
 struct BalancedLaunch {
   static constexpr size_t smem_bytes() {
-    return sizeof(BalancedSmem<G>) + 128;
+    return sizeof(BalancedSmem) + 1024;
   }
   static int ctas_per_sm() {
     static int occ = -1;  // per process; every B200 gives the same answer

@@ -265,10 +265,9 @@ static tv_status decode_common(void* out, float* partial_out,
                         (num_pages << shift) < (1 << 26) - 1 &&
                         (int64_t)num_seqs * num_kv_heads *
                                 (max_blocks_per_seq << shift) < INT32_MAX;
-  // the per-pair kernel reads its slices with ldmatrix from 128-byte
-  // swizzled boxes; the balanced kernel reads plain rows
-  const CUtensorMapSwizzle swz =
-      balanced ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+  // both decode kernels read their slices with ldmatrix from 128-byte
+  // swizzled boxes
+  const CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B;
   CUtensorMap tk, tvm;
   st = pool_tensor_map(&tk, k_pool, num_pages, page_size, num_kv_heads, swz);
   if (st != TV_OK) return st;
