@@ -190,3 +190,13 @@ def test_workspace_too_small_is_rejected():
     ws = _ws(db)
     with pytest.raises(_lib.TVError, match="INVALID_ARG"):
         _balanced(db, wl, ws[:1024], False)
+
+
+@pytest.mark.parametrize("scale", [-0.125, 0.0, 1.0])
+def test_scales_of_either_sign(scale):
+    """The balanced kernel scales each fp32 score before the maximum as
+    well: any finite scale, cut and uncut pairs, fused append."""
+    lens = [1, 16, 17, 300, 2049, 5000]
+    wl = W.decode_workload(lens, seed=302)
+    wl.scale = scale
+    _check(wl, True, f"balanced scale={scale}")

@@ -192,3 +192,29 @@ def test_fused_group_sizes(hq, hkv):
     ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
                               wl.scale)
     assert_parity(out, ref, f"fused hq={hq} hkv={hkv}")
+
+
+@pytest.mark.parametrize("scale", [-0.125, 0.0, 0.37, 1.0])
+def test_scales_of_either_sign(scale):
+    """Any finite scale (the decode scales each fp32 score before taking the
+    maximum): a negative one reverses the weights, 0 weighs every visible
+    key equally (the output is the mean of V), 1.0 makes the softmax peaked.
+    Plain and fused decode against the oracle at the same scale."""
+    lens = [1, 16, 17, 300, 2049]
+    wl = W.decode_workload(lens, seed=57)
+    wl.scale = scale
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, f"scale={scale}")
+    assert err_word(db) == 0
+    if scale == 0.0:
+        kp, vp = oracle_after_append(wl)
+        for s, n in enumerate(lens):
+            rows = [vp[wl.block_tables[s, t // 16], t % 16]
+                    for t in range(n)]
+            mean = np.mean(W.bf16_to_f64(np.stack(rows)), axis=0)  # [Hkv][D]
+            np.testing.assert_allclose(
+                W.bf16_to_f64(bf16_bits(out[s])),
+                np.repeat(mean, 4, axis=0), rtol=2**-7, atol=1e-3)
+    db2, fused = _fused(wl)
+    assert_parity(fused, ref, f"fused scale={scale}")
+    assert err_word(db2) == 0

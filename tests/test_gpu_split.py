@@ -43,6 +43,31 @@ def test_partials_match_oracle(pt):
     assert err_word(db) == 0
 
 
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 4)],
+                         ids=["mha", "gqa2", "gqa8"])
+def test_partials_group_sizes(hq, hkv):
+    """Split partials and the merge at every supported group size (the page
+    step pads the G heads of a KV head to the 8 columns of its products)."""
+    lens = [1, 17, 512, 513, 3000]
+    wl = W.decode_workload(lens, seed=25, num_q_heads=hq, num_kv_heads=hkv)
+    pt = 512
+    maxp = -(-max(lens) // pt) + 1
+    db = upload(wl)
+    gpu_append(db)
+    po, pl = gpu_split(db, wl.scale, pt, maxp)
+    out = gpu_merge(db, po, pl, pt)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ro, rl = oracle.paged_decode_partials(wl.q, kp, vp, wl.block_tables,
+                                          wl.context_lens, wl.scale, pt, maxp)
+    assert_parity(po, ro, f"o_p hq={hq} hkv={hkv}")
+    _lse_close(pl, rl, f"lse_p hq={hq} hkv={hkv}")
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, f"merged hq={hq} hkv={hkv}")
+    assert err_word(db) == 0
+
+
 def test_merge_kernel_matches_oracle_merge_on_the_same_partials():
     wl = W.decode_workload([100, 2000, 4097], seed=22)
     kp, vp = oracle_after_append(wl)
