@@ -41,12 +41,18 @@
 //      Warp 1 also allocates the tensor memory.
 //    warps 4-7 / 8-11: softmax of tile A / B.  Thread = one MMA row = one
 //      (query, head).  It reads its 64 scores from tensor memory in one load,
-//      takes their maximum, moves the running maximum only when it grows by
+//      moves the running maximum only when the tile's maximum exceeds it by
 //      more than 2^8 (then O and l are rescaled in place, which is rare, so O
 //      stays in tensor memory across key tiles), exponentiates, sums, and
 //      stores P_hi / P_lo into the same 64 columns (32 each, two bf16 per
-//      column).  The causal mask is applied only to the tiles that cross the
-//      diagonal.
+//      column).  After a row's first tile the running maximum is finite, so
+//      the warp exponentiates against it and takes the tile maximum in the
+//      same pass; only if some row's maximum grew by more than 2^8 does it
+//      reload the scores and redo the tile with the rescale (the result is
+//      the same either way: the offset rule does not change).  This removes
+//      the maximum from the path between the score load and the
+//      exponentials, the longest phase of the step after them.  The causal
+//      mask is applied only to the tiles that cross the diagonal.
 //  * P is split as P_hi = bf16(p), P_lo = bf16(p - P_hi) so the PV product
 //    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
 //    operands); a single bf16 P carries 8 bits, which is not enough for rows
@@ -432,14 +438,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       float s[kBN];
       tmem_ld64(s_addr + b * kBN, s);
       const uint32_t bad = sm.bad_pages[st];
-      if (!(full_tile && bad == 0)) {
+      const bool masked = !(full_tile && bad == 0);
+      auto apply_mask = [&]() {
 #pragma unroll
         for (int x = 0; x < kBN; ++x) {
           const int key = key0 + x;
           const bool vis = key <= limit && !((bad >> (x / kPS)) & 1u);
           s[x] = vis ? s[x] : -INFINITY;
         }
+      };
+      if (masked) apply_mask();
+
+      // packed fp32x2 arithmetic: one instruction per pair of keys
+      float2 lsum2 = make_float2(0.f, 0.f);
+      const float2 c2 = make_float2(c, c);
+      const float2 neg1 = make_float2(-1.f, -1.f);
+      uint32_t hi[kBN / 2], lo[kBN / 2];
+      // ---- after a row's first tile the running max is finite: exponentiate
+      //      against it while taking the tile maximum in the same pass; only
+      //      when a row's maximum grew by more than 2^8 is the tile redone
+      //      (S is still in tensor memory) with the rescale below ------------
+      bool exact = !__all_sync(0xffffffffu, m_run != -INFINITY);
+      if (!exact) {
+        float mx = -INFINITY;
+        const float2 nm2 = make_float2(-m_run, -m_run);
+#pragma unroll
+        for (int e = 0; e < kBN / 2; ++e) {
+          mx = fmax3(mx, s[2 * e], s[2 * e + 1]);
+          const float2 t = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), c2,
+                                      nm2);
+          const float2 x = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          lsum2 = __fadd2_rn(lsum2, x);
+          hi[e] = pack_bf16x2(x.x, x.y);
+          const float2 h = make_float2(bf16_lo(hi[e]), bf16_hi(hi[e]));
+          const float2 r = __ffma2_rn(h, neg1, x);   // x - hi, exact
+          lo[e] = pack_bf16x2(r.x, r.y);
+        }
+        exact = __any_sync(0xffffffffu, mx * c > m_run + kRescaleThreshold);
+        if (exact) {
+          tmem_ld64(s_addr + b * kBN, s);
+          if (masked) apply_mask();
+        }
       }
+      if (exact) {
       float mx = -INFINITY;
 #pragma unroll
       for (int x = 0; x < kBN; x += 2) mx = fmax3(mx, s[x], s[x + 1]);
@@ -470,12 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
 
       // ---- exponentials, row sum, P_hi / P_lo back into the S columns ------------
-      // packed fp32x2 arithmetic: one instruction per pair of keys
-      float2 lsum2 = make_float2(0.f, 0.f);
-      const float2 c2 = make_float2(c, c);
       const float2 nm2 = make_float2(-m_use, -m_use);
-      const float2 neg1 = make_float2(-1.f, -1.f);
-      uint32_t hi[kBN / 2], lo[kBN / 2];
+      lsum2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < kBN / 2; ++e) {
         const float2 t = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), c2,
@@ -486,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 h = make_float2(bf16_lo(hi[e]), bf16_hi(hi[e]));
         const float2 r = __ffma2_rn(h, neg1, x);   // x - hi, exact
         lo[e] = pack_bf16x2(r.x, r.y);
+      }
       }
       const float lsum = lsum2.x + lsum2.y;
       tmem_st32(s_addr + b * kBN, hi);
