@@ -97,3 +97,37 @@ def gpu_prefill(db, scale, max_query_len):
 def err_word(db) -> int:
     torch.cuda.synchronize()
     return int(db.err.item()) & 0xFFFFFFFF
+
+
+def grow_keys(wl, step=128, max_shift=6):
+    """Multiply the key row at position j of every sequence by
+    2^min(j // step, max_shift) (a power of two: exact in bf16), so the row
+    maxima of the scores climb along the context and the running offset of
+    the online softmax has to move again and again, far past the 2^8 the
+    kernels let it lag.  Cached keys are changed in the pool, the new
+    tokens' keys in k_new; stale slots keep their NaN poison."""
+    from paged_kv_cache_376_b200 import workloads as W
+    ps = wl.k_pool.shape[1]
+    new = np.diff(wl.query_start_loc)
+    cached = wl.context_lens - new
+    kp = wl.k_pool.reshape(-1, *wl.k_pool.shape[2:]).copy()
+    kn = wl.k_new.copy()
+
+    def scaled(bits, shift):
+        f = W.bf16_to_f64(bits) * (2.0 ** shift)[:, None, None]
+        return W.bf16_bits(f.astype(np.float32))
+
+    for s in range(wl.num_seqs):
+        pos = np.arange(int(cached[s]))
+        shift = np.minimum(pos // step, max_shift)
+        if len(pos):
+            slots = wl.block_tables[s, pos // ps].astype(np.int64) * ps + pos % ps
+            kp[slots] = scaled(kp[slots], shift)
+        q0 = int(wl.query_start_loc[s])
+        pos = int(cached[s]) + np.arange(int(new[s]))
+        if len(pos):
+            shift = np.minimum(pos // step, max_shift)
+            kn[q0:q0 + len(pos)] = scaled(kn[q0:q0 + len(pos)], shift)
+    wl.k_pool = kp.reshape(wl.k_pool.shape)
+    wl.k_new = kn
+    return wl

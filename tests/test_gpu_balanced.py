@@ -200,3 +200,12 @@ def test_scales_of_either_sign(scale):
     wl = W.decode_workload(lens, seed=302)
     wl.scale = scale
     _check(wl, True, f"balanced scale={scale}")
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["decode", "fused"])
+def test_growing_keys_move_the_running_maximum(fused):
+    """Keys scaled by 2^(position // 128): repeated rescales across pages,
+    in pairs cut over several ranges and merged by the last arriver."""
+    from gpu_util import grow_keys
+    wl = grow_keys(W.decode_workload([1, 130, 300, 1000, 4099, 6000], seed=303))
+    _check(wl, fused, f"balanced growing keys fused={fused}")

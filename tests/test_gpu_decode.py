@@ -218,3 +218,18 @@ def test_scales_of_either_sign(scale):
     db2, fused = _fused(wl)
     assert_parity(fused, ref, f"fused scale={scale}")
     assert err_word(db2) == 0
+
+
+def test_growing_keys_move_the_running_maximum():
+    """Keys scaled by 2^(position // 128) (up to 2^6): the page maxima keep
+    growing past the 2^8 lag the online softmax allows, so the accumulators
+    are rescaled again and again; plain and fused decode against the
+    oracle."""
+    from gpu_util import grow_keys
+    wl = grow_keys(W.decode_workload([1, 130, 300, 1000, 4099], seed=58))
+    db, out, ref = _run(wl)
+    assert_parity(out, ref, "growing keys")
+    assert err_word(db) == 0
+    db2, fused = _fused(wl)
+    assert_parity(fused, ref, "fused, growing keys")
+    assert err_word(db2) == 0

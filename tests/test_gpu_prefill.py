@@ -143,3 +143,18 @@ def test_cost_ordered_dispatch_is_bit_identical_to_grid_order():
                                wl.block_tables, wl.context_lens, wl.scale)
     assert_parity(outs[1], ref, "cost-ordered prefill")
     assert err_word(db) == 0
+
+
+def test_growing_keys_move_the_running_maximum():
+    """Keys scaled by 2^(position // 128) (up to 2^6): every row's maximum
+    keeps growing by far more than 2^8 over later key tiles, so the softmax
+    redoes tiles against the new maximum and rescales O in tensor memory,
+    repeatedly; every row against the oracle."""
+    from gpu_util import grow_keys
+    wl = grow_keys(W.prefill_workload([1000, 300, 0, 2000], [64, 200, 130, 48],
+                                      seed=35))
+    db, out, kp, vp = _run(wl)
+    ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp,
+                               wl.block_tables, wl.context_lens, wl.scale)
+    assert_parity(out, ref, "prefill, growing keys")
+    assert err_word(db) == 0

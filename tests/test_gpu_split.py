@@ -149,3 +149,28 @@ def test_long_split_config_every_row_partials_and_needles():
         got = bf16_bits(out[s, 8:12])
         np.testing.assert_array_equal(got, np.repeat(vp[page, off, 2][None],
                                                      4, axis=0))
+
+
+def test_growing_keys_partials_and_merge():
+    """Keys scaled by 2^(position // 128) (up to 2^6): partitions whose lse
+    differ by hundreds, and rescales inside each partition; partials and
+    the merged output against the oracle."""
+    from gpu_util import grow_keys
+    lens = [1, 300, 1000, 4099]
+    wl = grow_keys(W.decode_workload(lens, seed=26))
+    pt = 512
+    maxp = -(-max(lens) // pt)
+    db = upload(wl)
+    gpu_append(db)
+    po, pl = gpu_split(db, wl.scale, pt, maxp)
+    out = gpu_merge(db, po, pl, pt)
+    torch.cuda.synchronize()
+    kp, vp = oracle_after_append(wl)
+    ro, rl = oracle.paged_decode_partials(wl.q, kp, vp, wl.block_tables,
+                                          wl.context_lens, wl.scale, pt, maxp)
+    assert_parity(po, ro, "growing keys o_p")
+    _lse_close(pl, rl, "growing keys lse_p")
+    ref = oracle.paged_decode(wl.q, kp, vp, wl.block_tables, wl.context_lens,
+                              wl.scale)
+    assert_parity(out, ref, "growing keys merged")
+    assert err_word(db) == 0
