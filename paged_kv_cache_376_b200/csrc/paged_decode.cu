@@ -83,6 +83,22 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
   const int lane = threadIdx.x & 31;
   const int chk = lane & 7;    // 16-byte chunk of the appended row
 
+  // Block-table entries of this warp's first 64 blocks, loaded before and
+  // independently of the context length (bounded by the table row; entries
+  // past the context are loaded but never used), so the two loads overlap.
+  const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
+  const int sub_mask = (1 << a.page_shift) - 1;
+  const int first_page = kSplit ? part * a.partition_tokens / kPS : 0;
+  auto table_pid = [&](int i) -> int {
+    const int b = first_page + warp + kWarps * i;
+    if ((b >> a.page_shift) >= a.max_blocks_per_seq) return -1;
+    const int page = __ldg(bt + (b >> a.page_shift));
+    return page >= 0 && page < a.num_pages
+               ? (page << a.page_shift) + (b & sub_mask) : -1;
+  };
+  int pid_cur = table_pid(lane);
+  int pid_next = table_pid(32 + lane);
+
   // ---- token range of this CTA --------------------------------------------
   // a decode step (tv_decode_step) treats a sequence whose context did not
   // grow as idle: appending at ctx-1 would overwrite a cached token
@@ -102,12 +118,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     tok_end = min(ctx, tok_begin + a.partition_tokens);
     if (tok_end < tok_begin) tok_end = tok_begin;
   }
-  const int first_page = tok_begin / kPS;
   const int n_pages = (tok_end - tok_begin + kPS - 1) / kPS;
   // pages of this warp: first_page + warp + kWarps * i, i < my_n
   const int my_n = n_pages > warp ? (n_pages - warp + kWarps - 1) / kWarps : 0;
-  const int32_t* bt = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
-  const int sub_mask = (1 << a.page_shift) - 1;
 
   // ---- fused append: the new token is at position ctx-1 (unsplit kernel) ---
   int app_i = -1;            // local page index of the appended row, this warp
@@ -225,8 +238,6 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 4 : 2)
     return page >= 0 && page < a.num_pages
                ? (page << a.page_shift) + (b & sub_mask) : -1;
   };
-  int pid_cur = load_pids(0);
-  int pid_next = load_pids(1);
   const uint64_t policy = l2_policy_evict_first();
 
   auto issue = [&](int pid, int stage) {
