@@ -61,7 +61,31 @@ __global__ void __launch_bounds__(kThreads)
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
   if (M != -INFINITY) {
-    for (int p = pl; p < nparts; p += kPartLanes) {
+    // four partitions per lane in flight: the loads of a group are issued
+    // before any of them is used (the merge is bound by their latency)
+    constexpr int kU = 4;
+    int p = pl;
+    for (; p + (kU - 1) * kPartLanes < nparts; p += kU * kPartLanes) {
+      float l[kU];
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        l[u] = lse[p + u * kPartLanes];
+        v[u] = reinterpret_cast<const float4*>(
+            po + (size_t)(p + u * kPartLanes) * kD)[dq];
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const float w =
+            l[u] == -INFINITY ? 0.f : fast_exp2((l[u] - M) * kLog2e);
+        acc.x = fmaf(w, v[u].x, acc.x);
+        acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z);
+        acc.w = fmaf(w, v[u].w, acc.w);
+        wsum += w;
+      }
+    }
+    for (; p < nparts; p += kPartLanes) {
       const float l = lse[p];
       const float w = l == -INFINITY ? 0.f : fast_exp2((l - M) * kLog2e);
       const float4 v = reinterpret_cast<const float4*>(po + (size_t)p * kD)[dq];
