@@ -202,8 +202,10 @@ def split_merge(o_p, lse_p, context_lens, partition_tokens):
 
 
 def paged_prefill_rows(q, query_start_loc, k_pool, v_pool, block_tables,
-                       context_lens, scale, tok_idx, head_idx):
-    """Chunked-prefill attention for selected (query row, q-head) pairs."""
+                       context_lens, scale, tok_idx, head_idx, allow_bad=False):
+    """Chunked-prefill attention for selected (query row, q-head) pairs.
+    Keys whose page id is outside the pool are left out; that raises unless
+    ``allow_bad``."""
     lib = _load()
     q = _c(q, np.uint16)
     qsl = _c(query_start_loc, np.int32)
@@ -217,17 +219,18 @@ def paged_prefill_rows(q, query_start_loc, k_pool, v_pool, block_tables,
         _ptr(out), _ptr(ti), _ptr(hi), ti.shape[0], _ptr(q), _ptr(qsl),
         _ptr(kp), _ptr(vp), _ptr(bt), bt.shape[1], _ptr(cl),
         cl.shape[0], hq, hkv, d, page_size, num_pages, float(scale))
-    if bad:
+    if bad and not allow_bad:
         raise ValueError(f"{bad} keys referenced pages outside the pool")
     return out
 
 
 def paged_prefill(q, query_start_loc, k_pool, v_pool, block_tables,
-                  context_lens, scale):
+                  context_lens, scale, allow_bad=False):
     """Chunked-prefill attention for every row: float64 [rows][Hq][D]."""
     rows, hq, d = q.shape
     tok_idx = np.repeat(np.arange(rows, dtype=np.int32), hq)
     head_idx = np.tile(np.arange(hq, dtype=np.int32), rows)
     out = paged_prefill_rows(q, query_start_loc, k_pool, v_pool, block_tables,
-                             context_lens, scale, tok_idx, head_idx)
+                             context_lens, scale, tok_idx, head_idx,
+                             allow_bad=allow_bad)
     return out.reshape(rows, hq, d)

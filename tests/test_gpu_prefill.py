@@ -65,6 +65,33 @@ def test_chunked_prefill_config_every_row():
     assert_parity(out, ref, "chunked prefill, every row")
 
 
+def test_bad_page_ids_are_flagged_and_left_out():
+    """Block-table entries outside the pool: one in a cached prefix, one
+    under the first keys of a sequence with a prefix, and one covering every
+    key that the first 16 rows of a prefix-free sequence see (those rows
+    attend to nothing and come out zero).  The kernel flags the call and
+    leaves those keys out, as the oracle does with ``allow_bad``."""
+    from paged_kv_cache_376_b200 import _lib
+    wl = W.prefill_workload([100, 40, 0], [70, 30, 20], seed=37)
+    db = upload(wl)
+    gpu_append(db)                       # appended through the slot mapping
+    kp, vp = oracle_after_append(wl)
+    bt = wl.block_tables.copy()
+    bt[0, 2] = wl.num_pages + 5          # keys 32..47 of sequence 0
+    bt[1, 0] = -3                        # keys 0..15 of sequence 1
+    bt[2, 0] = wl.num_pages              # keys 0..15 of sequence 2
+    db.block_tables.copy_(torch.from_numpy(bt))
+    maxq = int(np.diff(wl.query_start_loc).max())
+    out = gpu_prefill(db, wl.scale, maxq)
+    torch.cuda.synchronize()
+    assert err_word(db) & _lib.DEVERR_BAD_PAGE
+    ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp, bt,
+                               wl.context_lens, wl.scale, allow_bad=True)
+    first = int(wl.query_start_loc[2])
+    assert not np.any(ref[first:first + 16])
+    assert_parity(out, ref, "prefill with bad page ids")
+
+
 def test_one_row_chunk_equals_decode():
     lens = [1, 40, 777]
     wl = W.prefill_workload([n - 1 for n in lens], [1] * len(lens), seed=32)
