@@ -162,18 +162,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                        uint32_t* err) {
   __shared__ int sh[33];
   __shared__ int job_old[kThreads], job_new[kThreads];
-  if (*p.page_size != kPS) {   // pools of another page size: touch nothing
-    if (threadIdx.x == 0) flag_error(err, DEVERR_BAD_SEQ);
-    if (threadIdx.x < num_seqs) p.grown[threadIdx.x] = 0;
-    return;
-  }
   const int s = threadIdx.x;
   const bool live = s < num_seqs;
-  int c = 0, n = 0, part = -1;
+  // The loads that do not depend on one another go out together (the kernel
+  // is a chain of dependent round trips: context -> last page -> its
+  // reference count -> free-stack pops); nothing below writes top or ref
+  // before the scans.
+  const int pool_ps = *p.page_size;
+  const int top = *p.top;
+  int c = live ? ctx[s] : 0;
+  int n = live && n_new ? n_new[s] : 0;
+  if (pool_ps != kPS) {   // pools of another page size: touch nothing
+    if (threadIdx.x == 0) flag_error(err, DEVERR_BAD_SEQ);
+    if (live) p.grown[s] = 0;
+    return;
+  }
+  int part = -1, r = 0;
   if (live) {
-    c = ctx[s];
     // decode steps (n_new == nullptr) add one token to every live sequence
-    n = n_new ? n_new[s] : (c > 0 ? 1 : 0);
+    if (!n_new) n = c > 0 ? 1 : 0;
     if (n < 0) n = 0;
     if (c < 0 || c + n > mb * kPS) {
       flag_error(err, DEVERR_BAD_CONTEXT);
@@ -188,19 +195,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         atomicAdd(p.cnt_app + part, 1);
         atomicMax(p.last_app + part, s + 1);
+        r = p.ref[part];
       }
     }
   }
   __syncthreads();
-  // copy-on-write decision (see the file comment) and pages needed
+  // copy-on-write decision (see the file comment) and pages needed; the
+  // writer counts are read only for a shared page
   bool cow = false;
-  if (part >= 0) {
-    const int r = p.ref[part];
-    cow = r > 1 && !(p.cnt_app[part] == r && p.last_app[part] == s + 1);
-  }
+  if (part >= 0 && r > 1)
+    cow = !(p.cnt_app[part] == r && p.last_app[part] == s + 1);
   const int need =
       n > 0 ? (int)cow + pages_for(c + n, kPS) - pages_for(c, kPS) : 0;
-  const int top = *p.top;
   int total;
   const int off = block_exclusive_scan(need, sh, &total);
   const bool served = live && n > 0 && off + need <= top;
