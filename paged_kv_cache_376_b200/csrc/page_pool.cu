@@ -66,8 +66,9 @@ __device__ __forceinline__ int pages_for(int ctx, int ps) {
   return (ctx + ps - 1) / ps;
 }
 
-// Exclusive scan of one int per thread over the 1024 threads of the CTA;
-// *total receives the sum.  `sh` holds 32 ints.
+// Exclusive scan of one int per thread over the threads of the CTA (a
+// multiple of 32, at most 1024); *total receives the sum.  `sh` holds 33
+// ints.
 __device__ int block_exclusive_scan(int v, int* sh, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
@@ -80,7 +81,7 @@ __device__ int block_exclusive_scan(int v, int* sh, int* total) {
   if (lane == 31) sh[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int w = sh[lane];
+    const int w = lane < (int)(blockDim.x >> 5) ? sh[lane] : 0;
     int wi = w;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int j = 0; j < njobs; ++j) {
     const size_t src = (size_t)jl_old[j] * kPS * row_bytes;
     const size_t dst = (size_t)jl_new[j] * kPS * row_bytes;
-    for (int v = threadIdx.x; v < page_vec; v += kThreads) {
+    for (int v = threadIdx.x; v < page_vec; v += blockDim.x) {
       reinterpret_cast<uint4*>(k_pool + dst)[v] =
           reinterpret_cast<const uint4*>(k_pool + src)[v];
       reinterpret_cast<uint4*>(v_pool + dst)[v] =
@@ -415,7 +416,10 @@ cudaError_t launch_pool_append(int32_t* state, int num_pages, int page_size,
                                int32_t* slot_mapping, void* k_pool,
                                void* v_pool, int row_bytes, uint32_t* err,
                                cudaStream_t stream) {
-  pool_append_kernel<<<1, kThreads, 0, stream>>>(
+  // one thread per sequence, whole warps (the scans' barriers are cheaper
+  // over fewer warps)
+  const int threads = num_seqs < 32 ? 32 : ((num_seqs + 31) / 32) * 32;
+  pool_append_kernel<<<1, threads < kThreads ? threads : kThreads, 0, stream>>>(
       view(state, num_pages), bt, mb, ctx, n_new, num_seqs, slot_mapping,
       static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool),
       row_bytes, page_size, err);
