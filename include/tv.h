@@ -312,13 +312,14 @@ tv_status tv_split_merge(void* out, const float* partial_out,
  *   query_start_loc  [num_seqs + 1] int32, non-decreasing, [0] == 0,
  *                    [num_seqs] <= num_query_rows
  *   max_query_len    >= every T_s (sizes the grid); rows beyond a
- *                    sequence's T_s are not touched; at most 65535 * 64
+ *                    sequence's T_s are not touched; at most 65535 blocks
+ *                    of 256 / G rows (G = num_q_heads / num_kv_heads)
  *   workspace        NULL, or device memory of at least
  *                    tv_prefill_workspace_size() bytes, 16-byte aligned, no
  *                    initial contents needed; too small or misaligned
  *                    returns TV_ERR_INVALID_ARG.  Given, a one-CTA kernel
- *                    first lists the work blocks (64 query rows of one
- *                    sequence) by their number of key tiles, costliest
+ *                    first lists the work blocks (256 / G query rows of
+ *                    one sequence) by their number of key tiles, costliest
  *                    first, and the attention grid runs them in that order,
  *                    so that long-context blocks do not start last and hold
  *                    a few SMs while the rest idle.  The results are the
@@ -326,7 +327,8 @@ tv_status tv_split_merge(void* out, const float* partial_out,
  *                    separate workspaces.
  *   workspace_bytes  its size
  * A sequence with T_s > C is flagged TV_DEVERR_BAD_QUERY and skipped.
- * Supported: num_q_heads == 4 * num_kv_heads (TV_ERR_UNSUPPORTED
+ * Supported: num_q_heads == G * num_kv_heads with G = 1, 2, 4 or 8 (one MMA
+ * tile = 128 / G query rows x the G heads of a KV head; TV_ERR_UNSUPPORTED
  * otherwise) and scale > 0 (TV_ERR_INVALID_ARG otherwise: the kernel takes
  * each key tile's maximum on the raw scores q.K and scales it afterwards,
  * which equals the maximum of the scaled scores only for a positive scale).
@@ -344,7 +346,9 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
 /*
  * tv_prefill_workspace_size -- bytes of the optional tv_paged_prefill
  * workspace for num_seqs sequences and the given max_query_len (4 bytes per
- * 64-row block of every sequence, rounded up to 16).
+ * 32-row block of every sequence, rounded up to 16: enough for every group
+ * size; a call checks the size its own group needs, 4 bytes per block of
+ * 256 / G rows).
  *   bytes   host pointer, written on TV_OK
  */
 tv_status tv_prefill_workspace_size(int num_seqs, int max_query_len,

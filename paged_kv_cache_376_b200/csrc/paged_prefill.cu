@@ -10,13 +10,14 @@
 // online softmax, tile sized to on-chip memory ("Tiny-vLLM 实战：用 C++/CUDA
 // 手写高性能 LLM 推理引擎", sec. "算子融合", FlashAttention-like blocking).
 //
-// B200 design (one CTA per (KV head, 64-query block, sequence); 12 warps):
-//  * An MMA tile has M = 128 rows = 32 query rows x the 4 query heads of one
-//    KV head, so every K/V tile feeds 4 heads (GQA reuse).  A CTA owns two
-//    such query tiles (A: rows q0..q0+31, B: q0+32..q0+63) that share every
-//    K/V tile, and the tensor core alternates between them while the other
-//    tile's softmax runs.  q arrives by one 3-D TMA box {64 d, 4 heads, 32
-//    rows} per tile.
+// B200 design (one CTA per (KV head, block of 256 / G query rows, sequence);
+// 12 warps; G = query heads per KV head, 1, 2, 4 or 8):
+//  * An MMA tile has M = 128 rows = 128 / G query rows x the G query heads of
+//    one KV head (32 x 4 for Llama-3.2-1B), so every K/V tile feeds G heads
+//    (GQA reuse).  A CTA owns two such query tiles (A, then B) that share
+//    every K/V tile, and the tensor core alternates between them while the
+//    other tile's softmax runs.  q arrives by one 3-D TMA box {64 d, G heads,
+//    128 / G rows} per tile; MMA row r is query row r / G, head r % G.
 //  * Keys come in tiles of 64 = 4 pages; each page of one KV head (16 rows x
 //    128 B) is one 2-D TMA box, 128-byte swizzled, so 4 boxes at 2 KB
 //    offsets form exactly the canonical K-major SW128 operand.  Pages past
@@ -58,8 +59,8 @@
 //    keeps ~16 bits of each weight (fp32-grade accumulation with bf16
 //    operands); a single bf16 P carries 8 bits, which is not enough for rows
 //    that see few keys.
-//  * With a workspace, a one-CTA kernel first lists the (sequence, 64-row
-//    block) items costliest first (cost = key tiles), and the attention grid
+//  * With a workspace, a one-CTA kernel first lists the (sequence, block)
+//    items costliest first (cost = key tiles), and the attention grid
 //    takes its work from that list, so that the longest blocks do not start
 //    last and hold a few SMs while the rest idle.
 //  * Every wait is an mbarrier wait bounded by a 2 s time limit.
@@ -71,10 +72,8 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kPS = 16;
-constexpr int kG = 4;                    // query heads per KV head
-constexpr int kQRows = 32;               // query rows per MMA tile
 constexpr int kQTiles = 2;               // MMA tiles per CTA (A, B)
-constexpr int kBM = kQRows * kG;         // 128 MMA rows
+constexpr int kBM = kPrefillTileRows;    // 128 MMA rows = (128 / G) query rows x G heads
 constexpr int kBN = 64;                  // keys per tile
 constexpr int kPagesPerTile = kBN / kPS; // 4
 constexpr int kST = 8;                   // K/V ring depth
@@ -122,10 +121,11 @@ __device__ __forceinline__ int prefill_cost(const PrefillArgs& a, int item,
   const int T = a.query_start_loc[seq + 1] - a.query_start_loc[seq];
   const int ctx = min(a.context_lens[seq],
                       a.max_blocks_per_seq * (kPS << a.page_shift));
-  const int q0 = blk * kPrefillRowsPerCta;
+  const int rows = prefill_rows_per_cta(a.group);
+  const int q0 = blk * rows;
   if (T <= 0 || q0 >= T || T > ctx) return 0;    // no work (or flagged)
   const int tiles =
-      (ctx - T + min(q0 + kPrefillRowsPerCta, T) + kBN - 1) / kBN;
+      (ctx - T + min(q0 + rows, T) + kBN - 1) / kBN;
   return min(tiles, kCostBuckets - 1);
 }
 
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kOrderThreads, 1)
     prefill_order_kernel(const PrefillArgs a) {
   __shared__ int slot[kCostBuckets];   // histogram, then next free position
   __shared__ int warp_sum[kOrderThreads / 32];
-  const int nblk = prefill_blocks(a.max_query_len);
+  const int nblk = prefill_blocks(a.max_query_len, a.group);
   const int n = a.num_seqs * nblk;
   for (int i = threadIdx.x; i < kCostBuckets; i += kOrderThreads) slot[i] = 0;
   __syncthreads();
@@ -178,11 +178,13 @@ __global__ void __launch_bounds__(kOrderThreads, 1)
     a.order[atomicAdd(&slot[prefill_cost(a, i, nblk)], 1)] = i;
 }
 
+template <int kG>   // query heads per KV head
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const PrefillArgs a,
                          const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
+  constexpr int kQRows = kBM / kG;         // query rows per MMA tile
   extern __shared__ __align__(1024) uint8_t smem_dyn[];
   uint8_t* base = smem_dyn + ((1024 - (smem_u32(smem_dyn) & 1023)) & 1023);
   auto& sm = *reinterpret_cast<PrefillSmem*>(base);
@@ -421,8 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;            // tensor-memory lane quarter
     const int r = quarter * 32 + lane;       // MMA row
     const int qt0 = q0 + t * kQRows;         // first chunk row of this tile
-    const int qi = r >> 2;                   // query row within the tile
-    const int hh = r & 3;                    // head within the group
+    const int qi = r / kG;                   // query row within the tile
+    const int hh = r % kG;                   // head within the group
     const bool row_real = qt0 + qi < T;
     const int limit = row_real ? P + qt0 + qi : ctx - 1;  // last visible key
     const int my_tiles = n_tiles_of[t];
@@ -603,18 +605,23 @@ cudaError_t launch_paged_prefill(const PrefillArgs& a, const CUtensorMap& tq,
                                  const CUtensorMap& tk, const CUtensorMap& tv,
                                  cudaStream_t stream) {
   const int smem = sizeof(PrefillSmem) + 1024;
+  auto kern = a.group == 1   ? paged_prefill_kernel<1>
+              : a.group == 2 ? paged_prefill_kernel<2>
+              : a.group == 8 ? paged_prefill_kernel<8>
+                             : paged_prefill_kernel<4>;
+  if (a.group != 1 && a.group != 2 && a.group != 4 && a.group != 8)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(
-      paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  static_assert(kQRows * kQTiles == kPrefillRowsPerCta, "rows per CTA");
   if (a.order) {
     prefill_order_kernel<<<1, kOrderThreads, 0, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const int blocks = prefill_blocks(a.max_query_len);
+  const int blocks = prefill_blocks(a.max_query_len, a.group);
   dim3 grid(a.num_kv_heads, blocks, a.num_seqs);
-  paged_prefill_kernel<<<grid, kThreads, smem, stream>>>(a, tq, tk, tv);
+  kern<<<grid, kThreads, smem, stream>>>(a, tq, tk, tv);
   return cudaGetLastError();
 }
 

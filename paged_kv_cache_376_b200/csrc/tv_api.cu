@@ -87,9 +87,10 @@ tv_status pool_tensor_map(CUtensorMap* map, const void* pool,
   return TV_OK;
 }
 
-// q seen as a 3-D bf16 tensor [rows][Hq][D]; the box is 32 rows x G heads x
-// 64 elements, i.e. the 4 query heads of one KV group for 32 query rows,
-// which land in shared memory as 128 rows of 128 B in (row, head) order.
+// q seen as a 3-D bf16 tensor [rows][Hq][D]; the box is rows_per_box rows x
+// G heads x 64 elements, i.e. the G query heads of one KV group for 128 / G
+// query rows, which land in shared memory as 128 rows of 128 B in (row,
+// head) order.
 tv_status query_tensor_map(CUtensorMap* map, const void* q, int64_t rows,
                            int num_q_heads, int group, int rows_per_box) {
   auto fn = encode_fn();
@@ -578,8 +579,13 @@ tv_status tv_split_merge(void* out, const float* partial_out,
       static_cast<cudaStream_t>(stream)));
 }
 
-static size_t prefill_workspace_bytes(int num_seqs, int max_query_len) {
-  const size_t items = (size_t)num_seqs * (size_t)tv::prefill_blocks(max_query_len);
+// Items of the ordering list: one per (sequence, block of
+// prefill_rows_per_cta(group) rows).  The size query has no group, so it
+// answers for the largest group (the most blocks).
+static size_t prefill_workspace_bytes(int num_seqs, int max_query_len,
+                                      int group = 8) {
+  const size_t items =
+      (size_t)num_seqs * (size_t)tv::prefill_blocks(max_query_len, group);
   return (items * sizeof(int32_t) + 15) / 16 * 16;
 }
 
@@ -602,7 +608,7 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   tv_status st =
       check_attention_shape(num_q_heads, num_kv_heads, head_dim, page_size);
   if (st != TV_OK) return st;
-  if (num_q_heads / num_kv_heads != 4) return TV_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;   // 1, 2, 4 or 8 (checked)
   // the kernel scales each tile's maximum raw score, which is the maximum
   // of the scaled scores only when the scale is positive
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_pages <= 0 ||
@@ -622,18 +628,19 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
     return TV_ERR_INVALID_ARG;
   if (workspace &&
       (!aligned16(workspace) ||
-       workspace_bytes < prefill_workspace_bytes(num_seqs, max_query_len)))
+       workspace_bytes <
+           prefill_workspace_bytes(num_seqs, max_query_len, group)))
     return TV_ERR_INVALID_ARG;
-  if (tv::prefill_blocks(max_query_len) > 65535) return TV_ERR_UNSUPPORTED;
+  if (tv::prefill_blocks(max_query_len, group) > 65535) return TV_ERR_UNSUPPORTED;
   // the ordering kernel counts the (sequence, block) items in an int
   if (workspace &&
-      (int64_t)num_seqs * tv::prefill_blocks(max_query_len) > INT32_MAX)
+      (int64_t)num_seqs * tv::prefill_blocks(max_query_len, group) > INT32_MAX)
     return TV_ERR_UNSUPPORTED;
 
   // Query rows past num_query_rows read as zeros and are never stored.
   CUtensorMap tq, tk, tvm;
-  st = query_tensor_map(&tq, q, num_query_rows, num_q_heads,
-                        num_q_heads / num_kv_heads, 32);
+  st = query_tensor_map(&tq, q, num_query_rows, num_q_heads, group,
+                        tv::kPrefillTileRows / group);
   if (st != TV_OK) return st;
   st = pool_tensor_map(&tk, k_pool, num_pages, page_size, num_kv_heads,
                        CU_TENSOR_MAP_SWIZZLE_128B);
@@ -658,6 +665,7 @@ tv_status tv_paged_prefill(void* out, const void* q, int64_t num_query_rows,
   a.scale_log2 = scale * 1.4426950408889634f;
   a.page_shift = page_shift(page_size);
   a.order = static_cast<int32_t*>(workspace);
+  a.group = group;
   return cuda_status(tv::launch_paged_prefill(
       a, tq, tk, tvm, static_cast<cudaStream_t>(stream)));
 }

@@ -122,15 +122,22 @@ struct PrefillArgs {
   int64_t num_query_rows;
   float scale_log2;
   int page_shift;                // page_size = 16 << page_shift
-  // Dispatch order: order[i] = seq * prefill_blocks(max_query_len) + block of
+  int group;                     // query heads per KV head: 1, 2, 4 or 8
+  // Dispatch order: order[i] = seq * prefill_blocks(max_query_len, group) + block of
   // the i-th CTA group (costliest first), written by the ordering kernel
   // into caller workspace; nullptr = grid order.
   int32_t* order;
 };
 
-constexpr int kPrefillRowsPerCta = 64;   // query rows (chunk positions) per CTA
-__host__ __device__ inline int prefill_blocks(int max_query_len) {
-  return (max_query_len + kPrefillRowsPerCta - 1) / kPrefillRowsPerCta;
+// A prefill CTA owns two MMA tiles of 128 rows = (128 / group) query rows x
+// the group's heads, so 256 / group query rows (chunk positions).
+constexpr int kPrefillTileRows = 128;
+__host__ __device__ inline int prefill_rows_per_cta(int group) {
+  return 2 * kPrefillTileRows / group;
+}
+__host__ __device__ inline int prefill_blocks(int max_query_len, int group) {
+  const int rows = prefill_rows_per_cta(group);
+  return (max_query_len + rows - 1) / rows;
 }
 
 // Launches the ordering kernel first when a.order is set.

@@ -65,8 +65,8 @@ def test_unsupported_shapes_are_rejected_before_launch(lib):
     assert lib.tv_kv_append(p, p, p, 4, p, p, 10, 8, 96, 16, None,
                             None) == 2
     assert lib.tv_split_merge(p, p, p, p, 2, 32, 32, 512, 4, None) == 2
-    # prefill needs 4 query heads per KV head
-    assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, 4, p, 1, 8, 8, 8, 64,
+    # prefill takes 1, 2, 4 or 8 query heads per KV head, not 16
+    assert lib.tv_paged_prefill(p, p, 8, p, p, p, p, 4, p, 1, 8, 32, 2, 64,
                                 16, 10, 0.1, None, 0, None, None) == 2
 
 
@@ -160,14 +160,28 @@ def test_sizes_beyond_32_bit_positions_are_refused(lib):
 def test_prefill_workspace_size(lib):
     import ctypes
     n = ctypes.c_size_t(0)
-    # 4 bytes per 64-row block of every sequence, rounded up to 16
+    # 4 bytes per 32-row block of every sequence (the blocks of the largest
+    # group size, 8: 256 / 8 rows), rounded up to 16
     assert lib.tv_prefill_workspace_size(3, 100, ctypes.byref(n)) == 0
-    assert n.value == 32          # 3 x 2 blocks = 24 bytes
+    assert n.value == 48          # 3 x 4 blocks = 48 bytes
     assert lib.tv_prefill_workspace_size(16, 512, ctypes.byref(n)) == 0
-    assert n.value == 512         # 16 x 8 blocks
+    assert n.value == 1024        # 16 x 16 blocks
     assert lib.tv_prefill_workspace_size(0, 0, ctypes.byref(n)) == 0
     assert n.value == 0
     assert lib.tv_prefill_workspace_size(-1, 8, ctypes.byref(n)) == 1
+
+
+def test_prefill_workspace_is_checked_for_the_call_group(lib):
+    """A call checks the workspace its own group needs: 16 sequences of up
+    to 512 rows need 16 x 8 blocks of 64 rows at G = 4 (512 bytes) but
+    16 x 16 blocks of 32 rows at G = 8 (1024 bytes)."""
+    p = _fake()
+    args = lambda hq, hkv, nbytes: (p, p, 8192, p, p, p, p, 64, p, 16, 512, hq,
+                                    hkv, 64, 16, 4096, 0.1, p, nbytes, None,
+                                    None)
+    assert lib.tv_paged_prefill(*args(32, 4, 512)) == 1      # G = 8: too small
+    assert lib.tv_paged_prefill(*args(32, 4, 1023)) == 1
+    assert lib.tv_paged_prefill(*args(24, 8, 64)) == 2       # G = 3: unsupported
 
 
 def test_empty_work_is_a_no_op(lib):

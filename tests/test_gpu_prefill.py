@@ -172,6 +172,39 @@ def test_cost_ordered_dispatch_is_bit_identical_to_grid_order():
     assert err_word(db) == 0
 
 
+@pytest.mark.parametrize("hq,hkv", [(32, 32), (32, 16), (32, 4), (64, 8)],
+                         ids=["gqa1", "gqa2", "gqa8", "gqa8-hq64"])
+def test_group_sizes_match_oracle_in_both_orders(hq, hkv):
+    """Group sizes 1, 2 and 8: an MMA tile is 128 / G query rows x G heads,
+    so a CTA covers 256 / G rows and the blocks, the ordering list and the
+    q boxes all change with G.  Ragged chunks over prefixes that are not
+    multiples of a tile; grid order and cost order give the same bits, and
+    both match the oracle on every (row, head)."""
+    from paged_kv_cache_376_b200 import _lib
+    wl = W.prefill_workload([0, 77, 300, 1000], [130, 45, 257, 9], seed=41,
+                            num_q_heads=hq, num_kv_heads=hkv)
+    db = upload(wl)
+    gpu_append(db)
+    maxq = int(np.diff(wl.query_start_loc).max())
+    outs = []
+    for ordered in (False, True):
+        out = torch.full_like(db.q, float("nan"))
+        ws = _lib.prefill_workspace(wl.num_seqs, maxq)
+        ws.fill_(0x5A)
+        _lib.tv_paged_prefill(out, db.q, db.query_start_loc, db.k_pool,
+                              db.v_pool, db.block_tables, db.context_lens,
+                              wl.scale, maxq, err=db.err, workspace=ws,
+                              ordered=ordered)
+        torch.cuda.synchronize()
+        outs.append(out)
+    np.testing.assert_array_equal(bf16_bits(outs[0]), bf16_bits(outs[1]))
+    kp, vp = oracle_after_append(wl)
+    ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp,
+                               wl.block_tables, wl.context_lens, wl.scale)
+    assert_parity(outs[0], ref, f"prefill hq={hq} hkv={hkv}")
+    assert err_word(db) == 0
+
+
 def test_growing_keys_move_the_running_maximum():
     """Keys scaled by 2^(position // 128) (up to 2^6): every row's maximum
     keeps growing by far more than 2^8 over later key tiles, so the softmax

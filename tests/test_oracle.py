@@ -282,7 +282,10 @@ def test_prefill_without_prefix_is_causal_self_attention():
 
 
 @pytest.mark.parametrize("hq,hkv,d,ps", [(32, 8, 64, 16), (32, 8, 64, 32),
-                                         (8, 2, 8, 4)])
+                                         (8, 2, 8, 4), (8, 8, 8, 4),
+                                         (8, 4, 8, 4), (16, 2, 8, 4)],
+                         ids=["gqa4", "gqa4-p32", "gqa4-small", "mha",
+                              "gqa2", "gqa8"])
 def test_prefill_with_prefix_matches_brute_force(hq, hkv, d, ps):
     rng = np.random.default_rng(23)
     prefixes, chunks = [0, 5, 33, 100], [3, 20, 16, 9]
