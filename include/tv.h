@@ -36,7 +36,7 @@
  *   - Supported: head_dim == 64, page_size 16 or 32 ([P3] recommends 16-32
  *     tokens; the kernels stream 16-token blocks, two per 32-token page),
  *     num_q_heads a multiple of num_kv_heads with a ratio in {1, 2, 4, 8}
- *     (tv_paged_prefill: 4 only); every pointer 16-byte aligned; num_seqs
+ *     (every call); every pointer 16-byte aligned; num_seqs
  *     <= 65535; num_pages * page_size and
  *     max_blocks_per_seq * page_size at most INT32_MAX (token positions and
  *     pool rows are 32-bit in the kernels).  Anything else returns
