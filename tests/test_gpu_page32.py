@@ -99,9 +99,12 @@ def test_balanced(fused):
     assert err_word(db) == 0
 
 
-def test_prefill():
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (32, 4), (16, 16)],
+                         ids=["gqa4", "gqa8", "mha"])
+def test_prefill(hq, hkv):
     wl = W.prefill_workload([0, 5, 16, 40, 1000, 333], [1, 31, 33, 64, 130, 17],
-                            seed=405, page_size=PS)
+                            seed=405, page_size=PS, num_q_heads=hq,
+                            num_kv_heads=hkv)
     db = upload(wl)
     gpu_append(db)
     maxq = int(np.diff(wl.query_start_loc).max())
@@ -110,7 +113,7 @@ def test_prefill():
     kp, vp = oracle_after_append(wl)
     ref = oracle.paged_prefill(wl.q, wl.query_start_loc, kp, vp,
                                wl.block_tables, wl.context_lens, wl.scale)
-    assert_parity(out, ref, "prefill PS32")
+    assert_parity(out, ref, f"prefill PS32 hq={hq} hkv={hkv}")
     assert err_word(db) == 0
 
 
